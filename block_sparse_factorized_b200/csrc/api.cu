@@ -1,0 +1,303 @@
+// api.cu -- C ABI entry points: argument checks, TMA descriptors, launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "kernels.h"
+#include "layout.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool encode(CUtensorMap *m, const void *base, CUtensorMapDataType dt, cuuint32_t rank,
+            const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box)
+{
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return encode_fn()(m, dt, rank, const_cast<void *>(base), dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of a bf16 [BH, n, 64] tensor in the natural, grid-column and summary frames.
+bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum)
+{
+    memset(&m, 0, sizeof(m));
+    const cuuint64_t row = 64 * 2, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
+    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    {
+        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[2] = {row, n * row};
+        const cuuint32_t box[3] = {64, 128, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box)) return false;
+    }
+    if (col) {
+        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[3] = {l * row, row, n * row};
+        const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(g.Rt), static_cast<cuuint32_t>(g.cpt), 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box)) return false;
+    }
+    if (sum) {
+        const cuuint64_t dims[4] = {64, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[3] = {row, l * row, n * row};
+        const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(g.c), static_cast<cuuint32_t>(g.upt), 1};
+        if (!encode(&m.sum, base, dt, 4, dims, str, box)) return false;
+    }
+    return true;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Frames {
+    bool qcol = false, kcol = false, ksum = false;
+};
+
+Frames frames_used(const st_layout &L)
+{
+    Frames f;
+    for (const auto &p : L.parts) {
+        f.qcol |= (p.qframe == st::FR_COL);
+        f.kcol |= (p.kframe == st::FR_COL);
+        f.ksum |= (p.kframe == st::FR_SUM);
+    }
+    return f;
+}
+
+st_status_t check_common(const st_layout *L, const st_desc_t *desc)
+{
+    if (!L || !desc) return ST_ERR_INVALID_ARG;
+    if (desc->reserved != 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
+        return ST_ERR_INVALID_ARG;
+    if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
+    if (desc->heads != L->pat.num_heads || desc->n != L->n) return ST_ERR_INVALID_ARG;
+    if (!L->exec_ok) return ST_ERR_UNSUPPORTED;
+    if (desc->d != 64) return ST_ERR_UNSUPPORTED;
+    if (desc->dtype != ST_BF16) return ST_ERR_UNSUPPORTED;
+    if (desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
+    if (!L->uploaded) return ST_ERR_NOT_UPLOADED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
+    if (dev != L->device) return ST_ERR_INVALID_ARG;
+    if (!encode_fn()) return ST_ERR_CUDA;
+    return ST_OK;
+}
+
+constexpr float LOG2E = 1.4426950408889634f;
+
+}  // namespace
+
+extern "C" {
+
+size_t st_attn_fwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
+{
+    (void)desc;
+    (void)layout;
+    return 0;
+}
+
+size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
+{
+    if (!desc || !layout) return 0;
+    const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
+    const size_t dq = rows * 64 * sizeof(float);
+    const size_t dl = rows * sizeof(float);
+    return ((dq + 255) & ~size_t(255)) + ((dl + 255) & ~size_t(255));
+}
+
+st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_layout_t *layout,
+                        void *o, float *lse, void *workspace, size_t workspace_bytes,
+                        const st_desc_t *desc, st_stream_t stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (!q || !k || !v || !o || !lse) return ST_ERR_INVALID_ARG;
+    const st_status_t cs = check_common(layout, desc);
+    if (cs != ST_OK) return cs;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ST_ERR_ALIGNMENT;
+    const st_layout &L = *layout;
+    const int64_t BH = desc->batch * desc->heads;
+    const Frames f = frames_used(L);
+    st::FwdParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) ||
+        !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.o, o, L.geom, BH, f.qcol, false))
+        return ST_ERR_CUDA;
+    p.parts = L.d_parts;
+    p.batch = static_cast<int32_t>(desc->batch);
+    p.heads = static_cast<int32_t>(desc->heads);
+    p.g = L.geom;
+    p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
+    p.lse = lse;
+    p.o_prev = static_cast<const uint16_t *>(o);
+    p.err = L.d_err;
+    for (int pass = 0; pass < 2; ++pass) {
+        p.items = L.d_fwd[pass];
+        p.nitems = static_cast<int32_t>(L.fwd_items[pass].size());
+        if (st::launch_fwd(p, stream) != cudaSuccess) return ST_ERR_CUDA;
+    }
+    return ST_OK;
+}
+
+namespace {
+
+struct BwdWs {
+    float *dq_acc, *delta;
+};
+
+st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void *workspace,
+                          size_t workspace_bytes, BwdWs &ws)
+{
+    if (!workspace || workspace_bytes < st_attn_bwd_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
+    const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
+    ws.dq_acc = static_cast<float *>(workspace);
+    ws.delta = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                         ((rows * 64 * sizeof(float) + 255) & ~size_t(255)));
+    return ST_OK;
+}
+
+}  // namespace
+
+st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t *layout, void *dk,
+                                void *dv, void *workspace, size_t workspace_bytes,
+                                const st_desc_t *desc, st_stream_t stream)
+{
+    if (!o || !dO || !dk || !dv) return ST_ERR_INVALID_ARG;
+    st_status_t cs = check_common(layout, desc);
+    if (cs != ST_OK) return cs;
+    BwdWs ws;
+    if ((cs = bwd_workspace(desc, layout, workspace, workspace_bytes, ws)) != ST_OK) return cs;
+    if (!aligned16(o) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv)) return ST_ERR_ALIGNMENT;
+    st::PreParams pre;
+    memset(&pre, 0, sizeof(pre));
+    pre.o = static_cast<const uint16_t *>(o);
+    pre.dout = static_cast<const uint16_t *>(dO);
+    pre.delta = ws.delta;
+    pre.dq_acc = ws.dq_acc;
+    pre.dk = static_cast<uint16_t *>(dk);
+    pre.dv = static_cast<uint16_t *>(dv);
+    pre.zero_fill = layout->d_zero_fill;
+    pre.rows = desc->batch * desc->heads * desc->n;
+    pre.n = static_cast<int32_t>(desc->n);
+    pre.heads = static_cast<int32_t>(desc->heads);
+    return st::launch_bwd_pre(pre, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+}
+
+st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
+                             const void *dO, const st_layout_t *layout, void *dk, void *dv,
+                             void *workspace, size_t workspace_bytes, const st_desc_t *desc,
+                             st_stream_t stream)
+{
+    if (!q || !k || !v || !lse || !dO || !dk || !dv) return ST_ERR_INVALID_ARG;
+    st_status_t cs = check_common(layout, desc);
+    if (cs != ST_OK) return cs;
+    BwdWs ws;
+    if ((cs = bwd_workspace(desc, layout, workspace, workspace_bytes, ws)) != ST_OK) return cs;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dk) || !aligned16(dv))
+        return ST_ERR_ALIGNMENT;
+    const st_layout &L = *layout;
+    const int64_t BH = desc->batch * desc->heads;
+    const Frames f = frames_used(L);
+    st::BwdParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dO, L.geom, BH, f.qcol, false) ||
+        !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) ||
+        !make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum))
+        return ST_ERR_CUDA;
+    p.parts = L.d_parts;
+    p.batch = static_cast<int32_t>(desc->batch);
+    p.heads = static_cast<int32_t>(desc->heads);
+    p.g = L.geom;
+    p.scale_log2 = LOG2E / 8.0f;
+    p.ds_scale = 1.0f / 8.0f;
+    p.lse = lse;
+    p.delta = ws.delta;
+    p.dq_acc = ws.dq_acc;
+    p.dk_prev = static_cast<const uint16_t *>(dk);
+    p.dv_prev = static_cast<const uint16_t *>(dv);
+    p.err = L.d_err;
+    for (int pass = 0; pass < 2; ++pass) {
+        p.items = L.d_bwd[pass];
+        p.nitems = static_cast<int32_t>(L.bwd_items[pass].size());
+        if (st::launch_bwd(p, stream) != cudaSuccess) return ST_ERR_CUDA;
+    }
+    return ST_OK;
+}
+
+st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *workspace,
+                               size_t workspace_bytes, const st_desc_t *desc, st_stream_t stream)
+{
+    if (!dq) return ST_ERR_INVALID_ARG;
+    st_status_t cs = check_common(layout, desc);
+    if (cs != ST_OK) return cs;
+    BwdWs ws;
+    if ((cs = bwd_workspace(desc, layout, workspace, workspace_bytes, ws)) != ST_OK) return cs;
+    if (!aligned16(dq)) return ST_ERR_ALIGNMENT;
+    st::ConvParams cv;
+    cv.dq_acc = ws.dq_acc;
+    cv.dq = static_cast<uint16_t *>(dq);
+    cv.elems = desc->batch * desc->heads * desc->n * 64;
+    return st::launch_dq_convert(cv, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+}
+
+st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                        const float *lse, const void *dO, const st_layout_t *layout, void *dq,
+                        void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                        const st_desc_t *desc, st_stream_t stream)
+{
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ST_ERR_INVALID_ARG;
+    st_status_t cs = check_common(layout, desc);
+    if (cs != ST_OK) return cs;
+    BwdWs ws;
+    if ((cs = bwd_workspace(desc, layout, workspace, workspace_bytes, ws)) != ST_OK) return cs;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return ST_ERR_ALIGNMENT;
+    if ((cs = st_attn_bwd_prepare(o, dO, layout, dk, dv, workspace, workspace_bytes, desc, stream)) != ST_OK)
+        return cs;
+    if ((cs = st_attn_bwd_main(q, k, v, lse, dO, layout, dk, dv, workspace, workspace_bytes, desc,
+                               stream)) != ST_OK)
+        return cs;
+    return st_attn_bwd_finish(layout, dq, workspace, workspace_bytes, desc, stream);
+}
+
+const char *st_status_string(st_status_t s)
+{
+    switch (s) {
+    case ST_OK: return "ok";
+    case ST_ERR_INVALID_ARG: return "invalid argument";
+    case ST_ERR_UNSUPPORTED: return "unsupported by the kernels";
+    case ST_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case ST_ERR_NOT_UPLOADED: return "layout not uploaded";
+    case ST_ERR_CUDA: return "CUDA error";
+    case ST_ERR_OOM: return "out of memory";
+    case ST_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case ST_ERR_WORKSPACE: return "workspace missing or too small";
+    case ST_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+const char *st_version(void) { return "st_attn 0.1 (sm_100a)"; }
+
+}  // extern "C"

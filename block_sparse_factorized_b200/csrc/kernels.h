@@ -1,0 +1,69 @@
+// kernels.h -- parameter blocks and launch wrappers of the sm_100a kernels (internal).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "frames.cuh"
+
+namespace st {
+
+// Tensor maps of one [B*H, n, 64] tensor in the three frames (see frames.cuh):
+//   nat: dims {64, n, BH},       box {64, 128, 1}
+//   col: dims {64, R, l, BH},    box {64, Rt, cpt, 1}   (grid view, read column-wise)
+//   sum: dims {64, l, R, BH},    box {64, c, 128/c, 1}  (summary runs of each block)
+struct FrameMaps {
+    CUtensorMap nat, col, sum;
+};
+
+struct FwdParams {
+    FrameMaps q, k, v, o;        // o.sum unused
+    const Part *parts;
+    const WorkItem *items;
+    int32_t nitems, batch, heads;
+    Geom g;
+    float scale_log2;            // log2(e) / sqrt(d)
+    float *lse;                  // [B*H, n]
+    const uint16_t *o_prev;      // merge pass: the output (bf16) written by the first pass
+    int32_t *err;                // device error word
+};
+
+struct BwdParams {
+    FrameMaps q, k, v, dout;
+    FrameMaps dk, dv;            // stores (sum used for compacted keys)
+    const Part *parts;
+    const WorkItem *items;
+    int32_t nitems, batch, heads;
+    Geom g;
+    float scale_log2;            // log2(e) / sqrt(d)
+    float ds_scale;              // 1 / sqrt(d), folded into dS
+    const float *lse;            // [B*H, n] natural-log lse of the forward
+    const float *delta;          // [B*H, n] D_i = dO_i . O_i
+    float *dq_acc;               // [B*H, n, 64] fp32, zeroed before the main kernel
+    const uint16_t *dk_prev;     // merge pass: dK, dV written by the first pass (bf16)
+    const uint16_t *dv_prev;
+    int32_t *err;
+};
+
+struct PreParams {
+    const uint16_t *o, *dout;    // bf16 [B*H, n, 64]
+    float *delta;                // [B*H, n]
+    float *dq_acc;               // [B*H, n, 64] zeroed here
+    uint16_t *dk, *dv;           // zero-filled for heads flagged in zero_fill
+    const int32_t *zero_fill;    // [H]
+    int64_t rows;                // B*H*n
+    int32_t n, heads;
+};
+
+struct ConvParams {
+    const float *dq_acc;
+    uint16_t *dq;
+    int64_t elems;
+};
+
+cudaError_t launch_fwd(const FwdParams &p, cudaStream_t s);
+cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s);
+cudaError_t launch_bwd_pre(const PreParams &p, cudaStream_t s);
+cudaError_t launch_dq_convert(const ConvParams &p, cudaStream_t s);
+
+}  // namespace st

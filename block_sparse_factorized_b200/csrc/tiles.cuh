@@ -1,0 +1,65 @@
+// tiles.cuh -- frame-aware TMA tile transfers and fast exp2/log2, shared by the kernels.
+#pragma once
+#include "frames.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace st {
+
+constexpr uint32_t TILE_BYTES = 128 * 64 * 2;  // one 128 x 64 bf16 tile, 16 KB
+constexpr float LN2 = 0.6931471805599453f;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// Hardware base-2 exponential / logarithm (MUFU ex2 / lg2), flush-to-zero.
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ const CUtensorMap *frame_map(const FrameMaps &m, int32_t fr)
+{
+    return fr == FR_NAT ? &m.nat : (fr == FR_COL ? &m.col : &m.sum);
+}
+
+// TMA load of tile t of frame fr (summary offset o) of batch-head bh into dst (16 KB).
+__device__ __forceinline__ void load_tile(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
+                                          int32_t t, int32_t bh, void *dst, uint64_t *bar)
+{
+    if (fr == FR_NAT) {
+        tma_load_3d(dst, &m.nat, bar, 0, t * TILE, bh);
+    } else if (fr == FR_COL) {
+        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
+        tma_load_4d(dst, &m.col, bar, 0, rt * TILE, grp * g.cpt, bh);
+    } else {
+        tma_load_4d(dst, &m.sum, bar, 0, g.l - g.c - o, t * g.upt, bh);
+    }
+}
+
+// TMA store of a 16 KB tile; rows outside the tensor (padding of the grid and summary frames)
+// are clipped by the copy engine.
+__device__ __forceinline__ void store_tile(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
+                                           int32_t t, int32_t bh, const void *src)
+{
+    if (fr == FR_NAT) {
+        tma_store_3d(&m.nat, src, 0, t * TILE, bh);
+    } else if (fr == FR_COL) {
+        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
+        tma_store_4d(&m.col, src, 0, rt * TILE, grp * g.cpt, bh);
+    } else {
+        tma_store_4d(&m.sum, src, 0, g.l - g.c - o, t * g.upt, bh);
+    }
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+}  // namespace st

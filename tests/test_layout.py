@@ -1,0 +1,210 @@
+"""Host-side checks of the C ABI library (no GPU): exports, argument errors, and the block layout.
+
+* The library loads and exports every function include/st_attn.h declares.
+* Invalid arguments give the documented status codes, with no crash.
+* Natural-frame CSR + element masks expand, row by row, to exactly the oracle's allowed sets
+  (bit-exact), for every head of every workload and for small sweeps; FULL blocks are exactly the
+  blocks whose every pair is allowed; no empty block is listed.
+* The execution frames (natural, grid-column, compacted summary) enumerate, per row, exactly the
+  oracle's allowed set, using the same interval and frame rules as the kernels.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+bsf = pytest.importorskip("block_sparse_factorized_b200")
+from block_sparse_factorized_b200 import _abi  # noqa: E402
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "st_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(st_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _abi.load()
+    names = header_functions()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(_abi.EXPORTED)
+    assert b"sm_100a" in lib.st_version()
+    assert lib.st_status_string(0) == b"ok"
+
+
+def _build(family, mode, H, n, l, c=0, block=128, step=0):
+    lib = _abi.load()
+    h = ctypes.c_void_p()
+    pat = _abi.st_pattern_t(family, mode, H, step)
+    st = lib.st_layout_build(ctypes.byref(pat), n, l, c, block, ctypes.byref(h))
+    if st == 0:
+        lib.st_layout_destroy(h)
+    return st
+
+
+def test_argument_errors():
+    S, F, A = bsf.ST_STRIDED, bsf.ST_FIXED, bsf.ST_PER_HEAD_ALTERNATING
+    assert _build(S, A, 2, 256, 16) == 0
+    assert _build(3, A, 2, 256, 16) == 1          # bad family
+    assert _build(S, 9, 2, 256, 16) == 1          # bad head mode
+    assert _build(S, A, 0, 256, 16) == 1          # no heads
+    assert _build(S, A, 2, 0, 16) == 1            # n
+    assert _build(S, A, 2, 256, 0) == 1           # l
+    assert _build(S, A, 2, 256, 16, block=96) == 1
+    assert _build(F, A, 2, 256, 16, c=0) == 1     # fixed needs 1 <= c <= l
+    assert _build(F, A, 2, 256, 16, c=17) == 1
+    lib = _abi.load()
+    assert lib.st_layout_build(None, 256, 16, 0, 128, None) == 1
+    # a layout the kernels cannot run (n % 128 != 0) still builds and exports, but cannot upload
+    lay = bsf.Layout(S, A, 2, 200, 10)
+    rp, ci, mi, mk = lay.export(0)
+    assert rp[-1] == len(ci)
+    assert lib.st_layout_upload(lay.handle, None) == 2
+    with pytest.raises(bsf.StError):
+        lay.info()
+    # calls on a layout that was never uploaded: argument errors first, then NOT_UPLOADED
+    lay = bsf.Layout(S, A, 2, 256, 16)
+    fake = ctypes.c_void_p(1 << 20)
+    d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
+    assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 4
+    d = _abi.st_desc_t(1, 2, 256, 32, 1, 0)
+    assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 2
+    d = _abi.st_desc_t(1, 3, 256, 64, 1, 0)      # heads mismatch
+    assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
+    d = _abi.st_desc_t(1, 2, 256, 64, 7, 0)      # bad dtype
+    assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
+    d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
+    assert lib.st_attn_fwd(None, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
+    assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
+                           ctypes.byref(d), None) == 4
+    assert lib.st_layout_check(lay.handle, None) == 4
+
+
+def expand_block_row(row_ptr, col_idx, mask_id, masks, qb, B, n):
+    """Dense [B, n] allowed matrix of query block qb from the exported CSR."""
+    out = np.zeros((B, n), dtype=bool)
+    for e in range(row_ptr[qb], row_ptr[qb + 1]):
+        kb, m = col_idx[e], mask_id[e]
+        if m < 0:
+            blk = np.ones((B, B), dtype=bool)
+        else:
+            bits = np.unpackbits(masks[m].view(np.uint8), bitorder="little")
+            blk = bits.reshape(B, B).astype(bool)
+        assert blk.any(), "an empty block is listed"
+        cols = slice(kb * B, min(n, kb * B + B))
+        out[:, cols] |= blk[:, : cols.stop - cols.start]
+        if m >= 0:
+            assert not blk.all(), "a FULL block is stored with a mask"
+    return out
+
+
+def oracle_block_row(kind, o, qb, B, n, l, c):
+    out = np.zeros((B, n), dtype=bool)
+    for r in range(B):
+        i = qb * B + r
+        if i < n:
+            out[r, oracle.row_set(kind, i, l, c, o)] = True
+    return out
+
+
+def check_layout_bitexact(lay, n, l, c, qblocks=None):
+    B = lay.block
+    seen = set()
+    for h in range(lay.num_heads):
+        kind, o = lay.head_kind(h)
+        if (kind, o) in seen:
+            continue
+        seen.add((kind, o))
+        row_ptr, col_idx, mask_id, masks = lay.export(h)
+        nqb = (n + B - 1) // B
+        assert len(row_ptr) == nqb + 1
+        blocks = range(nqb) if qblocks is None else qblocks
+        for qb in blocks:
+            got = expand_block_row(row_ptr, col_idx, mask_id, masks, qb, B, n)
+            want = oracle_block_row(kind, o, qb, B, n, l, c)
+            assert np.array_equal(got, want), (kind, o, qb)
+            # a block is listed iff it holds an allowed pair
+            listed = set(col_idx[row_ptr[qb]:row_ptr[qb + 1]].tolist())
+            active = {j // B for j in np.nonzero(want.any(axis=0))[0]}
+            assert listed == active
+        assert len(set(map(bytes, masks))) == len(masks), "masks are not deduplicated"
+
+
+SWEEP = [  # (family, mode, H, n, l, c, block)
+    (1, 1, 2, 256, 16, 0, 64), (1, 1, 2, 256, 16, 0, 128), (1, 2, 3, 384, 24, 0, 64),
+    (1, 3, 1, 200, 7, 0, 64), (1, 4, 1, 200, 7, 0, 128), (2, 1, 8, 512, 64, 16, 64),
+    (2, 2, 4, 384, 32, 8, 128), (2, 4, 3, 300, 20, 5, 64), (2, 1, 4, 256, 256, 32, 128),
+]
+
+
+@pytest.mark.parametrize("cfg", SWEEP)
+def test_natural_csr_bitexact_sweep(cfg):
+    fam, mode, H, n, l, c, B = cfg
+    lay = bsf.Layout(fam, mode, H, n, l, c, block=B)
+    check_layout_bitexact(lay, n, l, c)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_natural_csr_bitexact_workloads(name):
+    w = WORKLOADS[name]
+    B = 64 if w.dtype == "fp32" else 128
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c, block=B)
+    nqb = w.n // B
+    qbl = None if nqb <= 96 else sorted(set(np.linspace(0, nqb - 1, 24).astype(int).tolist()))
+    check_layout_bitexact(lay, w.n, w.l, w.c, qbl)
+
+
+EXEC_SWEEP = [  # (family, mode, H, n, l, c) -- kernel-runnable layouts, every row checked
+    (1, 1, 2, 256, 16, 0), (1, 2, 2, 256, 16, 0), (1, 1, 2, 384, 3, 0), (1, 2, 2, 384, 3, 0),
+    (1, 1, 2, 512, 2, 0), (1, 2, 2, 256, 1, 0), (1, 1, 2, 256, 256, 0), (1, 2, 2, 768, 4, 0),
+    (2, 1, 8, 512, 128, 32), (2, 2, 4, 512, 128, 32), (2, 1, 4, 1024, 256, 8),
+    (2, 2, 4, 768, 64, 16), (2, 4, 4, 384, 128, 128), (1, 1, 2, 3072, 64, 0),
+    (1, 2, 2, 3072, 64, 0), (1, 1, 2, 32768, 256, 0),
+]
+
+
+@pytest.mark.parametrize("cfg", EXEC_SWEEP)
+def test_exec_frames_match_sets(cfg):
+    fam, mode, H, n, l, c = cfg
+    lay = bsf.Layout(fam, mode, H, n, l, c)
+    rows = range(n) if n <= 1024 else sorted(set(np.linspace(0, n - 1, 160).astype(int).tolist()))
+    for h in range(H):
+        kind, o = lay.head_kind(h)
+        for i in rows:
+            got = lay.exec_row(h, i)
+            want = oracle.row_set(kind, i, l, c, o)
+            assert np.array_equal(got, want), (cfg, h, i)
+
+
+def test_exec_tile_counts():
+    """Active 128 x 128 tile pairs the kernels compute, per batch element."""
+    w = WORKLOADS["fixed_n12288_l128_c32"]
+    info = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+    assert info["exec_tiles"] == 5184          # 4 x 96 (same block) + 4 x 1200 (summary)
+    assert info["allowed_pairs"] == 78673920   # sum of |A(h, i)| over heads and rows
+    assert info["passes"] == 1
+    w = WORKLOADS["strided_n12288_l128"]
+    info = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+    assert info["exec_tiles"] == 2552
+    w = WORKLOADS["strided_merged_n12288_l128"]
+    info = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+    assert info["exec_tiles"] == 5104 and info["passes"] == 2
+    w = WORKLOADS["strided_n65536_l256"]
+    info = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+    assert info["exec_tiles"] == 9204
+    for name, wl in WORKLOADS.items():
+        info = bsf.Layout(wl.family, wl.head_mode, wl.heads, wl.n, wl.l, wl.c).info()
+        kinds = [oracle.head_kinds(wl.family, wl.head_mode, wl.heads, wl.l, wl.c)]
+        total = 0
+        for kd, off in zip(*kinds[0]):
+            total += int(oracle.set_counts(int(kd), wl.n, wl.l, wl.c, int(off)).sum())
+        assert info["allowed_pairs"] == total, name
