@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of factorized sparse attention (forward + recomputing backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the workload: the fused forward
+kernel, then the backward pass's three phases (D_i and accumulator set-up, the recomputing
+tcgen05 kernel, dQ conversion).  The layout is built and uploaded once, outside the timed region.
+Inputs are seeded synthetic tensors (workloads.py), resident in HBM when timing starts; L2 is
+flushed (a 256 MiB write) before every timed step, outside the step's CUDA events.
+
+The metric counts active-block FLOPs: every 128 x 128 tile pair the kernels compute contributes
+128 * 128 * 4 * d FLOPs to the forward and 2.5 times that to the backward (five matmuls, one of
+them the recomputation of S), 3.5x in total.  `value` is the whole-job figure over all ranks
+(replicas: every rank runs the full workload on its own GPU; time is the max over ranks).
+
+The reference arm (--impl reference) is the fp64 CPU oracle, run on the host cores on a bounded
+sample of the workload per step and scaled to the metric's unit by the share of the workload it
+covered.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "active-block TFLOP/s fwd+bwd (bf16) at n=12288 and % of B200 tensor peak"
+UNIT = "TFLOP/s"
+TILE = 128
+FLUSH_BYTES = 256 << 20
+
+# DRAM traffic of the dominant kernel (st_attn_bwd_main) per launch, from an ncu capture, valid
+# only while the kernel sources hash to `src`.  Filled in from profiles/ after a capture.
+NCU_TRAFFIC = {}
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_factorized_b200", "csrc")
+    for name in ("bwd.cu", "tiles.cuh", "sm100.cuh", "frames.cuh", "kernels.h"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job(per_rank_units: float, times_s, world: int):
+    """Aggregate of replicas: all ranks' units over the slowest rank's time."""
+    return per_rank_units * world / max(times_s)
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+class ClockSampler:
+    """NVML samples of SM clock, power and throttle reasons every ~2 ms on a thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                uuid = None
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.h, self.ok = pynvml, h, True
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((mhz, reasons, pw))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = [name for b, name in self.REASONS.items() if bits & b]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------- oracle sample (CPU)
+def oracle_sample(w, slabs):
+    """Run the oracle's full forward + backward on the given (batch, head) slabs; return
+    (seconds, threads).  Each slab is one (b, h): the oracle runs the whole n for that head."""
+    import oracle
+    q, k, v, do = make_inputs(w)
+    kinds, offs = oracle.head_kinds(w.family, w.head_mode, w.heads, w.l, w.c, w.offset_step)
+    t0 = time.perf_counter()
+    for b, h in slabs:
+        p = oracle.Problem.from_kinds([kinds[h]], [offs[h]], w.l, w.c)
+        sl = [t[b:b + 1, h:h + 1].double().numpy() for t in (q, k, v, do)]
+        p.fwd(*sl[:3])
+        p.bwd(*sl)
+    return time.perf_counter() - t0, oracle.num_threads()
+
+
+def step_flops(w, info):
+    tiles = info["exec_tiles"] * w.batch
+    fwd = tiles * TILE * TILE * 4 * w.d
+    return fwd * 3.5, fwd * 2.5, info["allowed_pairs"] * w.batch * 4 * w.d * 3.5
+
+
+def layout_info_host(w):
+    import block_sparse_factorized_b200 as bsf
+    return bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return 0
+    info = layout_info_host(w)
+    flops, _, _ = step_flops(w, info)
+    slabs_all = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    per_step = []
+    threads = 1
+    for s in range(args.warmup + args.steps):
+        slab = slabs_all[s % len(slabs_all)] if w.head_mode == 2 else (0, s % w.heads)
+        secs, threads = oracle_sample(w, [slab])
+        if s >= args.warmup:
+            per_step.append(secs * len(slabs_all))   # time the whole workload would take
+    ms = 1e3 * statistics.mean(per_step)
+    value = flops / (ms / 1e3) / 1e12
+    sample = (f"oracle fwd+bwd of one (batch, head) slab per step (cycling heads), full n="
+              f"{w.n}; scaled by {len(slabs_all)} slabs")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "pattern": "fixed" if w.family == 2 else "strided",
+            "heads_mode": {1: "alternating", 2: "merged", 3: "head1", 4: "head2"}[w.head_mode],
+            "n": w.n, "l": w.l, "c": w.c, "batch": w.batch, "heads": w.heads, "d": w.d,
+            "io_dtype": w.dtype, "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    import block_sparse_factorized_b200 as bsf
+    from block_sparse_factorized_b200 import _abi
+    import ctypes
+
+    w = WORKLOADS[args.workload]
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).upload(stream)
+    info = lay.info()
+    flops, bwd_flops, useful = step_flops(w, info)
+    q, k, v, do = (t.to(device) for t in make_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    lib = _abi.load()
+    desc = bsf._desc(q)
+    ws_bytes = int(lib.st_attn_bwd_workspace_bytes(ctypes.byref(desc), lay.handle))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    P = ctypes.c_void_p
+
+    def ptr(t):
+        return P(t.data_ptr())
+
+    def fwd():
+        _abi.check(lib.st_attn_fwd(ptr(q), ptr(k), ptr(v), lay.handle, ptr(o), ptr(lse), None, 0,
+                                   ctypes.byref(desc), sp), "st_attn_fwd")
+
+    def prep():
+        _abi.check(lib.st_attn_bwd_prepare(ptr(o), ptr(do), lay.handle, ptr(dk), ptr(dv), ptr(ws),
+                                           ws_bytes, ctypes.byref(desc), sp), "st_attn_bwd_prepare")
+
+    def main():
+        _abi.check(lib.st_attn_bwd_main(ptr(q), ptr(k), ptr(v), ptr(lse), ptr(do), lay.handle,
+                                        ptr(dk), ptr(dv), ptr(ws), ws_bytes, ctypes.byref(desc), sp),
+                   "st_attn_bwd_main")
+
+    def finish():
+        _abi.check(lib.st_attn_bwd_finish(lay.handle, ptr(dq), ptr(ws), ws_bytes,
+                                          ctypes.byref(desc), sp), "st_attn_bwd_finish")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd(); prep(); main(); finish()
+    torch.cuda.synchronize(device)
+    lay.check(stream)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with sampler:
+        for s in range(args.steps):
+            flush.zero_()
+            e = ev[s]
+            e[0].record(stream); fwd(); e[1].record(stream); prep(); e[2].record(stream)
+            main(); e[3].record(stream); finish(); e[4].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    lay.check(stream)
+    t_step = [e[0].elapsed_time(e[4]) for e in ev]
+    t_fwd = [e[0].elapsed_time(e[1]) for e in ev]
+    t_prep = [e[1].elapsed_time(e[2]) for e in ev]
+    t_main = [e[2].elapsed_time(e[3]) for e in ev]
+    t_fin = [e[3].elapsed_time(e[4]) for e in ev]
+    ms_local = statistics.mean(t_step)
+    ms = max_over_ranks(ms_local, world, device)
+    value = flops * world / (ms / 1e3) / 1e12
+    launches_per_step = 2 * info["passes"] + 2
+    peaks = measured_peaks()
+    main_ms = statistics.mean(t_main)
+    achieved = bwd_flops / (main_ms / 1e3) / 1e12
+    src = kernel_src_hash()
+    tr = NCU_TRAFFIC.get((w.name, src))
+    roofline = {"kernel": "st_attn_bwd_main (bwd_kernel)", "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": tr, "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, lay, device, stream, flops, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        slabs = [(0, h) for h in range(min(2, w.heads))]
+        secs, threads = oracle_sample(w, slabs)
+        scale = (w.batch * w.heads) / len(slabs)
+        cpu_val = flops / (secs * scale) / 1e12
+        cpu = {"value": cpu_val, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"oracle fwd+bwd of batch 0, heads 0-{len(slabs) - 1} (full n={w.n}), "
+                         f"{secs:.1f} s, scaled by {scale:g} to the whole workload"}
+
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w),
+        "pct_of_tensor_peak": 100.0 * (value / world) / peaks["bf16_tflops"],
+        "useful_tflops": useful * world / (ms / 1e3) / 1e12,
+        "breakdown_ms": {"fwd": statistics.mean(t_fwd), "bwd_prepare": statistics.mean(t_prep),
+                         "bwd_main": main_ms, "bwd_finish": statistics.mean(t_fin)},
+        "fwd_tflops": flops / 3.5 / (statistics.mean(t_fwd) / 1e3) / 1e12,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        "exec_tiles": info["exec_tiles"] * w.batch, "kernel_src": src,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del lay
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, w, lay, device, stream, flops, world):
+    """Same metric through the public API with pinned host buffers: H2D of q, k, v, dO and D2H
+    of dq, dk, dv inside every timed step."""
+    import block_sparse_factorized_b200 as bsf
+    hq, hk, hv, hdo = (t.pin_memory() for t in make_inputs(w))
+    dq_h, dk_h, dv_h = (torch.empty_like(hq).pin_memory() for _ in range(3))
+    dev = [torch.empty_like(hq, device=device) for _ in range(4)]
+    o = torch.empty_like(dev[0])
+    lse = torch.empty(hq.shape[:3], dtype=torch.float32, device=device)
+    g = [torch.empty_like(dev[0]) for _ in range(3)]
+    ws = torch.empty(max(256, bsf.st_attn_bwd_workspace_bytes(dev[0], lay)), dtype=torch.uint8,
+                     device=device)
+
+    def step():
+        for d_, h_ in zip(dev, (hq, hk, hv, hdo)):
+            d_.copy_(h_, non_blocking=True)
+        bsf.st_attn_fwd(dev[0], dev[1], dev[2], lay, o=o, lse=lse, stream=stream)
+        bsf.st_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], lay, dq=g[0], dk=g[1], dv=g[2],
+                        workspace=ws, stream=stream)
+        for h_, d_ in zip((dq_h, dk_h, dv_h), g):
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, device)
+    nbytes = hq.numel() * hq.element_size()
+    return {"value": flops * world / (ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes,
+            "api": "block_sparse_factorized_b200.st_attn_fwd / st_attn_bwd (C ABI), pinned host buffers"}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device; this benchmark times the B200 kernels"}))
+        return 1
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
