@@ -90,7 +90,6 @@ st_status_t check_common(const st_layout *L, const st_desc_t *desc)
     if (desc->heads != L->pat.num_heads || desc->n != L->n) return ST_ERR_INVALID_ARG;
     if (!L->exec_ok) return ST_ERR_UNSUPPORTED;
     if (desc->d != 64) return ST_ERR_UNSUPPORTED;
-    if (desc->dtype != ST_BF16) return ST_ERR_UNSUPPORTED;
     if (desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
     if (!L->uploaded) return ST_ERR_NOT_UPLOADED;
     int dev = -1;
@@ -102,15 +101,32 @@ st_status_t check_common(const st_layout *L, const st_desc_t *desc)
 
 constexpr float LOG2E = 1.4426950408889634f;
 
+size_t bf16_copy_bytes(const st_desc_t *desc)
+{
+    const size_t b = static_cast<size_t>(desc->batch) * desc->heads * desc->n * 64 * 2;
+    return (b + 255) & ~size_t(255);
+}
+
+// fp32 I/O: round src to bf16 (and its residual) in the workspace.
+bool split_copy(const void *src, void *hi, void *lo, const st_desc_t *desc, st_stream_t stream)
+{
+    st::SplitParams sp;
+    sp.src = static_cast<const float *>(src);
+    sp.hi = static_cast<uint16_t *>(hi);
+    sp.lo = static_cast<uint16_t *>(lo);
+    sp.elems = desc->batch * desc->heads * desc->n * 64;
+    return st::launch_split(sp, stream) == cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t st_attn_fwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    (void)desc;
-    (void)layout;
-    return 0;
+    if (!desc || !layout || desc->dtype != ST_FP32) return 0;
+    // fp32 I/O: bf16 copies Q_hi, Q_lo, K_hi, K_lo, V_hi
+    return 5 * bf16_copy_bytes(desc);
 }
 
 size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
@@ -119,15 +135,15 @@ size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *lay
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
     const size_t dq = rows * 64 * sizeof(float);
     const size_t dl = rows * sizeof(float);
-    return ((dq + 255) & ~size_t(255)) + ((dl + 255) & ~size_t(255));
+    const size_t base = ((dq + 255) & ~size_t(255)) + ((dl + 255) & ~size_t(255));
+    // fp32 I/O adds bf16 copies of Q, K, V and dO for the tensor-core operands
+    return desc->dtype == ST_FP32 ? base + 4 * bf16_copy_bytes(desc) : base;
 }
 
 st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_layout_t *layout,
                         void *o, float *lse, void *workspace, size_t workspace_bytes,
                         const st_desc_t *desc, st_stream_t stream)
 {
-    (void)workspace;
-    (void)workspace_bytes;
     if (!q || !k || !v || !o || !lse) return ST_ERR_INVALID_ARG;
     const st_status_t cs = check_common(layout, desc);
     if (cs != ST_OK) return cs;
@@ -136,11 +152,28 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
     const st_layout &L = *layout;
     const int64_t BH = desc->batch * desc->heads;
     const Frames f = frames_used(L);
+    const bool f32 = desc->dtype == ST_FP32;
     st::FwdParams p;
     memset(&p, 0, sizeof(p));
-    if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) ||
-        !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.o, o, L.geom, BH, f.qcol, false))
+    if (f32) {
+        const size_t need = st_attn_fwd_workspace_bytes(desc, layout), cb = bf16_copy_bytes(desc);
+        if (!workspace || workspace_bytes < need) return ST_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
+        char *w = static_cast<char *>(workspace);
+        void *qh = w, *ql = w + cb, *kh = w + 2 * cb, *kl = w + 3 * cb, *vh = w + 4 * cb;
+        if (!split_copy(q, qh, ql, desc, stream) || !split_copy(k, kh, kl, desc, stream) ||
+            !split_copy(v, vh, nullptr, desc, stream))
+            return ST_ERR_CUDA;
+        if (!make_maps(p.q, qh, L.geom, BH, f.qcol, false) || !make_maps(p.ql, ql, L.geom, BH, f.qcol, false) ||
+            !make_maps(p.k, kh, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.kl, kl, L.geom, BH, f.kcol, f.ksum) ||
+            !make_maps(p.v, vh, L.geom, BH, f.kcol, f.ksum))
+            return ST_ERR_CUDA;
+        p.o_f32 = static_cast<float *>(o);
+        p.o_prev_f32 = static_cast<const float *>(o);
+    } else if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) ||
+               !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.o, o, L.geom, BH, f.qcol, false)) {
         return ST_ERR_CUDA;
+    }
     p.parts = L.d_parts;
     p.batch = static_cast<int32_t>(desc->batch);
     p.heads = static_cast<int32_t>(desc->heads);
@@ -152,7 +185,7 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
     for (int pass = 0; pass < 2; ++pass) {
         p.items = L.d_fwd[pass];
         p.nitems = static_cast<int32_t>(L.fwd_items[pass].size());
-        if (st::launch_fwd(p, stream) != cudaSuccess) return ST_ERR_CUDA;
+        if (st::launch_fwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
     return ST_OK;
 }
@@ -161,6 +194,7 @@ namespace {
 
 struct BwdWs {
     float *dq_acc, *delta;
+    char *copies;  // fp32 I/O: bf16 Q, K, V, dO
 };
 
 st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void *workspace,
@@ -172,6 +206,7 @@ st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void
     ws.dq_acc = static_cast<float *>(workspace);
     ws.delta = reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                          ((rows * 64 * sizeof(float) + 255) & ~size_t(255)));
+    ws.copies = reinterpret_cast<char *>(ws.delta) + ((rows * sizeof(float) + 255) & ~size_t(255));
     return ST_OK;
 }
 
@@ -189,8 +224,15 @@ st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t
     if (!aligned16(o) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv)) return ST_ERR_ALIGNMENT;
     st::PreParams pre;
     memset(&pre, 0, sizeof(pre));
+    const bool f32 = desc->dtype == ST_FP32;
     pre.o = static_cast<const uint16_t *>(o);
     pre.dout = static_cast<const uint16_t *>(dO);
+    if (f32) {
+        pre.o_f32 = static_cast<const float *>(o);
+        pre.dout_f32 = static_cast<const float *>(dO);
+        pre.dk_f32 = static_cast<float *>(dk);
+        pre.dv_f32 = static_cast<float *>(dv);
+    }
     pre.delta = ws.delta;
     pre.dq_acc = ws.dq_acc;
     pre.dk = static_cast<uint16_t *>(dk);
@@ -199,7 +241,7 @@ st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t
     pre.rows = desc->batch * desc->heads * desc->n;
     pre.n = static_cast<int32_t>(desc->n);
     pre.heads = static_cast<int32_t>(desc->heads);
-    return st::launch_bwd_pre(pre, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+    return st::launch_bwd_pre(pre, f32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
 st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
@@ -220,9 +262,27 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
     const Frames f = frames_used(L);
     st::BwdParams p;
     memset(&p, 0, sizeof(p));
-    if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dO, L.geom, BH, f.qcol, false) ||
-        !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) ||
-        !make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum))
+    const bool f32 = desc->dtype == ST_FP32;
+    const void *qb = q, *kb = k, *vb = v, *dob = dO;
+    if (f32) {
+        const size_t cb = bf16_copy_bytes(desc);
+        char *c = ws.copies;
+        if (!split_copy(q, c, nullptr, desc, stream) || !split_copy(k, c + cb, nullptr, desc, stream) ||
+            !split_copy(v, c + 2 * cb, nullptr, desc, stream) || !split_copy(dO, c + 3 * cb, nullptr, desc, stream))
+            return ST_ERR_CUDA;
+        qb = c;
+        kb = c + cb;
+        vb = c + 2 * cb;
+        dob = c + 3 * cb;
+        p.dk_f32 = static_cast<float *>(dk);
+        p.dv_f32 = static_cast<float *>(dv);
+        p.dk_prev_f32 = static_cast<const float *>(dk);
+        p.dv_prev_f32 = static_cast<const float *>(dv);
+    }
+    if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false) ||
+        !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum))
+        return ST_ERR_CUDA;
+    if (!f32 && (!make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum)))
         return ST_ERR_CUDA;
     p.parts = L.d_parts;
     p.batch = static_cast<int32_t>(desc->batch);
@@ -239,7 +299,7 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
     for (int pass = 0; pass < 2; ++pass) {
         p.items = L.d_bwd[pass];
         p.nitems = static_cast<int32_t>(L.bwd_items[pass].size());
-        if (st::launch_bwd(p, stream) != cudaSuccess) return ST_ERR_CUDA;
+        if (st::launch_bwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
     return ST_OK;
 }
@@ -256,8 +316,9 @@ st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *worksp
     st::ConvParams cv;
     cv.dq_acc = ws.dq_acc;
     cv.dq = static_cast<uint16_t *>(dq);
+    cv.dq_f32 = static_cast<float *>(dq);
     cv.elems = desc->batch * desc->heads * desc->n * 64;
-    return st::launch_dq_convert(cv, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+    return st::launch_dq_convert(cv, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
 st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void *o,

@@ -43,6 +43,8 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
+// F32: fp32 I/O -- dK and dV are written row by row in fp32 (the MMAs run on bf16 copies).
+template <bool F32>
 __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -252,6 +254,28 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 32; ++e) acc[h * 32 + e] = __uint_as_float(sv[e]);
                 }
+                if (F32) {
+                    if (pos >= 0 && *abort == 0) {
+                        const float *pf = which == 0 ? p.dk_prev_f32 : p.dv_prev_f32;
+                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64;
+                        if (part.merge) {
+                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                const float4 u = src[q];
+                                acc[4 * q] += u.x;
+                                acc[4 * q + 1] += u.y;
+                                acc[4 * q + 2] += u.z;
+                                acc[4 * q + 3] += u.w;
+                            }
+                        }
+                        float4 *d4 = reinterpret_cast<float4 *>(of);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            d4[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                    }
+                    continue;
+                }
                 if (part.merge && pos >= 0) {
                     const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64);
 #pragma unroll
@@ -275,7 +299,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             fence_proxy_async_smem();
         }
         named_bar_sync(1, 128);
-        if (row == 0 && ok && *abort == 0) {
+        if (!F32 && row == 0 && ok && *abort == 0) {
             store_tile(p.dk, part.kframe, p.g, part.o, kt, bh, smem + OFF_P);
             store_tile(p.dv, part.kframe, p.g, part.o, kt, bh, smem + OFF_P + TB);
             bulk_commit();
@@ -290,20 +314,26 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     }
 }
 
-}  // namespace
-
-cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s)
+template <bool F32>
+cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(bwd_kernel<F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (p.nitems == 0) return cudaSuccess;
-    bwd_kernel<<<dim3(static_cast<unsigned>(p.nitems) * p.batch), THREADS, SMEM_BYTES, s>>>(p);
+    bwd_kernel<F32><<<dim3(static_cast<unsigned>(p.nitems) * p.batch), THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s)
+{
+    return f32 ? launch_bwd_t<true>(p, s) : launch_bwd_t<false>(p, s);
 }
 
 }  // namespace st

@@ -3,27 +3,36 @@
 //                whose keys are not all written by the main kernel (fixed pattern-2 heads read
 //                only summary positions; every other key gets no gradient).
 //   dq_convert:  dQ fp32 accumulator -> output dtype (round to nearest even).
+//   split:       fp32 tensor -> bf16 high part (round to nearest even) and optionally the bf16
+//                low part x - hi, the operands of the split-precision products of fp32 I/O.
 // Both are HBM-bound: 8 threads per 64-wide row, 16-byte accesses, grid sized to the SM count.
-#include "kernels.h"
-#include "sm100.cuh"
+#include "tiles.cuh"
 
 namespace st {
 namespace {
 
-__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
+template <bool F32>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p)
 {
-    const int64_t sub = threadIdx.x & 7;  // 16-byte slice of the row (8 bf16)
+    const int64_t sub = threadIdx.x & 7;  // eighth of the 64-wide row
     const int64_t nthr_rows = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 3);
     for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 3) + (threadIdx.x >> 3);
          r < p.rows; r += nthr_rows) {
-        const uint4 a = reinterpret_cast<const uint4 *>(p.o + r * 64)[sub];
-        const uint4 b = reinterpret_cast<const uint4 *>(p.dout + r * 64)[sub];
-        float s = bf_lo(a.x) * bf_lo(b.x) + bf_hi(a.x) * bf_hi(b.x) + bf_lo(a.y) * bf_lo(b.y) +
-                  bf_hi(a.y) * bf_hi(b.y) + bf_lo(a.z) * bf_lo(b.z) + bf_hi(a.z) * bf_hi(b.z) +
-                  bf_lo(a.w) * bf_lo(b.w) + bf_hi(a.w) * bf_hi(b.w);
+        float s;
+        if (F32) {
+            const float4 *a = reinterpret_cast<const float4 *>(p.o_f32 + r * 64) + 2 * sub;
+            const float4 *b = reinterpret_cast<const float4 *>(p.dout_f32 + r * 64) + 2 * sub;
+            const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+            s = a0.x * b0.x + a0.y * b0.y + a0.z * b0.z + a0.w * b0.w + a1.x * b1.x + a1.y * b1.y +
+                a1.z * b1.z + a1.w * b1.w;
+        } else {
+            const uint4 a = reinterpret_cast<const uint4 *>(p.o + r * 64)[sub];
+            const uint4 b = reinterpret_cast<const uint4 *>(p.dout + r * 64)[sub];
+            s = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
+                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
+                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+        }
         s += __shfl_xor_sync(0xffffffffu, s, 1);
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         s += __shfl_xor_sync(0xffffffffu, s, 4);
@@ -33,12 +42,19 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p)
         acc[2 * sub + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
         const int32_t h = static_cast<int32_t>((r / p.n) % p.heads);
         if (p.zero_fill[h]) {
-            reinterpret_cast<uint4 *>(p.dk + r * 64)[sub] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4 *>(p.dv + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+            if (F32) {
+                float4 *k4 = reinterpret_cast<float4 *>(p.dk_f32 + r * 64) + 2 * sub;
+                float4 *v4 = reinterpret_cast<float4 *>(p.dv_f32 + r * 64) + 2 * sub;
+                k4[0] = k4[1] = v4[0] = v4[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                reinterpret_cast<uint4 *>(p.dk + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4 *>(p.dv + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+            }
         }
     }
 }
 
+template <bool F32>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const ConvParams p)
 {
     const int64_t n8 = p.elems / 8;
@@ -46,8 +62,35 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const ConvParams p)
          a += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float4 x = reinterpret_cast<const float4 *>(p.dq_acc)[2 * a];
         const float4 y = reinterpret_cast<const float4 *>(p.dq_acc)[2 * a + 1];
-        reinterpret_cast<uint4 *>(p.dq)[a] =
+        if (F32) {
+            reinterpret_cast<float4 *>(p.dq_f32)[2 * a] = x;
+            reinterpret_cast<float4 *>(p.dq_f32)[2 * a + 1] = y;
+        } else {
+            reinterpret_cast<uint4 *>(p.dq)[a] = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w),
+                                                            pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+        }
+    }
+}
+
+__device__ __forceinline__ float bf16_round(float x) { return bf16_lo(pack_bf16(x, 0.f)); }
+
+__global__ void __launch_bounds__(256) split_kernel(const SplitParams p)
+{
+    const int64_t n8 = p.elems / 8;
+    for (int64_t a = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; a < n8;
+         a += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 x = reinterpret_cast<const float4 *>(p.src)[2 * a];
+        const float4 y = reinterpret_cast<const float4 *>(p.src)[2 * a + 1];
+        reinterpret_cast<uint4 *>(p.hi)[a] =
             make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+        if (p.lo) {
+            const float v[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+            float r[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = v[e] - bf16_round(v[e]);
+            reinterpret_cast<uint4 *>(p.lo)[a] = make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]),
+                                                            pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7]));
+        }
     }
 }
 
@@ -65,21 +108,35 @@ int sm_count()
 
 }  // namespace
 
-cudaError_t launch_bwd_pre(const PreParams &p, cudaStream_t s)
+int blocks_for(int64_t work_units)
 {
-    const int64_t want = (p.rows + 31) / 32;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    const int blocks = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
-    bwd_pre_kernel<<<blocks, 256, 0, s>>>(p);
+    return static_cast<int>(work_units < cap ? (work_units > 0 ? work_units : 1) : cap);
+}
+
+cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s)
+{
+    const int blocks = blocks_for((p.rows + 31) / 32);
+    if (f32)
+        bwd_pre_kernel<true><<<blocks, 256, 0, s>>>(p);
+    else
+        bwd_pre_kernel<false><<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_dq_convert(const ConvParams &p, cudaStream_t s)
+cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s)
 {
-    const int64_t want = (p.elems / 8 + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    const int blocks = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
-    dq_convert_kernel<<<blocks, 256, 0, s>>>(p);
+    const int blocks = blocks_for((p.elems / 8 + 255) / 256);
+    if (f32)
+        dq_convert_kernel<true><<<blocks, 256, 0, s>>>(p);
+    else
+        dq_convert_kernel<false><<<blocks, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split(const SplitParams &p, cudaStream_t s)
+{
+    split_kernel<<<blocks_for((p.elems / 8 + 255) / 256), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

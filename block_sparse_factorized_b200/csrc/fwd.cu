@@ -23,14 +23,23 @@ namespace {
 
 constexpr int NST = 2;                         // K/V ring depth
 constexpr uint32_t TB = TILE_BYTES;            // one 128 x 64 bf16 tile, 16 KB
-constexpr uint32_t OFF_Q = 0;                  // also the O staging tile in the epilogue
-constexpr uint32_t OFF_K = OFF_Q + TB;
-constexpr uint32_t OFF_V = OFF_K + NST * TB;
-constexpr uint32_t OFF_P = OFF_V + NST * TB;   // P as two 128 x 64 halves (keys 0-63, 64-127)
-constexpr uint32_t OFF_BAR = OFF_P + 2 * TB;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 256;            // S: columns 0..127, O: 128..191
+
+// Shared-memory plan.  SPLIT (fp32 I/O) adds the low bf16 parts of Q and of each K tile.
+//   Q [, Q_lo] | NST x (K, V [, K_lo]) | P (two 128 x 64 halves: keys 0-63, 64-127) | barriers
+// The Q tile doubles as the O staging tile of the epilogue.
+template <bool SPLIT>
+struct Plan {
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_QL = TB;
+    static constexpr uint32_t OFF_STAGE = (SPLIT ? 2 : 1) * TB;
+    static constexpr uint32_t STAGE = (SPLIT ? 3 : 2) * TB;     // K at +0, V at +TB, K_lo at +2TB
+    static constexpr uint32_t OFF_P = OFF_STAGE + NST * STAGE;
+    static constexpr uint32_t OFF_BAR = OFF_P + 2 * TB;
+    static constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+    static constexpr int MIN_BLOCKS = SPLIT ? 1 : 2;
+};
 
 struct Bars {
     uint64_t q_full, s_full, p_full, o_done;
@@ -40,8 +49,12 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 128, "barrier block");
 
-__global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__ FwdParams p)
+template <bool SPLIT>
+__global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
+    fwd_kernel(const __grid_constant__ FwdParams p)
 {
+    using L = Plan<SPLIT>;
+    constexpr uint32_t OFF_Q = L::OFF_Q, OFF_P = L::OFF_P, OFF_BAR = L::OFF_BAR;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BAR);
@@ -84,18 +97,22 @@ __global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__
             tma_prefetch(frame_map(mq, part.qframe));
             tma_prefetch(frame_map(mk, part.kframe));
             tma_prefetch(frame_map(mv, part.kframe));
-            mbar_arrive_expect_tx(&bars->q_full, TB);
+            mbar_arrive_expect_tx(&bars->q_full, (SPLIT ? 2 : 1) * TB);
             load_tile(mq, part.qframe, p.g, part.o, w.tile, bh, smem + OFF_Q, &bars->q_full);
+            if (SPLIT)
+                load_tile(p.ql, part.qframe, p.g, part.o, w.tile, bh, smem + L::OFF_QL, &bars->q_full);
             int it = 0;
             for (; it < nkt; ++it) {
                 const int s = it % NST;
                 if (it >= NST && !mbar_wait(&bars->kv_empty[s], ((it / NST) - 1) & 1, abort, p.err))
                     break;
-                mbar_arrive_expect_tx(&bars->kv_full[s], 2 * TB);
-                load_tile(mk, part.kframe, p.g, part.o, w.begin + it, bh, smem + OFF_K + s * TB,
-                          &bars->kv_full[s]);
-                load_tile(mv, part.kframe, p.g, part.o, w.begin + it, bh, smem + OFF_V + s * TB,
-                          &bars->kv_full[s]);
+                uint8_t *stage = smem + L::OFF_STAGE + s * L::STAGE;
+                mbar_arrive_expect_tx(&bars->kv_full[s], L::STAGE);
+                load_tile(mk, part.kframe, p.g, part.o, w.begin + it, bh, stage, &bars->kv_full[s]);
+                load_tile(mv, part.kframe, p.g, part.o, w.begin + it, bh, stage + TB, &bars->kv_full[s]);
+                if (SPLIT)
+                    load_tile(p.kl, part.kframe, p.g, part.o, w.begin + it, bh, stage + 2 * TB,
+                              &bars->kv_full[s]);
             }
             if (*abort) {  // drain the copies still in flight before the CTA leaves
                 volatile int32_t never = 0;
@@ -116,13 +133,24 @@ __global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__
                     const int s = it % NST;
                     if (!mbar_wait(&bars->kv_full[s], (it / NST) & 1, abort, p.err)) break;
                     tc_fence_after();
-                    const uint32_t sK = smem_u32(smem + OFF_K + s * TB);
-                    const uint32_t sV = smem_u32(smem + OFF_V + s * TB);
-                    // S = Q K^T: both operands K-major, 16 elements (32 bytes) of d per step
+                    const uint32_t sK = smem_u32(smem + L::OFF_STAGE + s * L::STAGE);
+                    const uint32_t sV = sK + TB;
+                    // S = Q K^T: both operands K-major, 16 elements (32 bytes) of d per step.
+                    // Split precision adds Q_hi K_lo^T + Q_lo K_hi^T into the same accumulator.
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
                                     desc_sw128(sK + 32 * k, 16, 1024), idS, k > 0 ? 1u : 0u);
+                    if (SPLIT) {
+                        const uint32_t sQl = smem_u32(smem + L::OFF_QL), sKl = sK + 2 * TB;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
+                                        desc_sw128(sKl + 32 * k, 16, 1024), idS, 1u);
+                            mma_bf16_ss(tS, desc_sw128(sQl + 32 * k, 16, 1024),
+                                        desc_sw128(sK + 32 * k, 16, 1024), idS, 1u);
+                        }
+                    }
                     mma_commit(&bars->s_full);
                     if (!mbar_wait(&bars->p_full, it & 1, abort, p.err)) break;
                     tc_fence_after();
@@ -237,13 +265,9 @@ __global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__
         float w2 = has ? 1.f / l : 0.f;                     // weight of this part's acc
         float lse2 = has ? m + lg2(l) : -INFINITY;          // log2 units
         float w1 = 0.f;
-        uint4 prev[8];
         const size_t rowoff = (static_cast<size_t>(bh) * p.g.n + (i < 0 ? 0 : i));
         if (part.merge && i >= 0) {
             const float L1 = p.lse[rowoff] * LOG2E;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * 64);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) prev[j] = src[j];
             const float Lm = fmaxf(L1, lse2);
             if (Lm == -INFINITY) {
                 w2 = 0.f;
@@ -256,29 +280,56 @@ __global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__
             }
         }
         if (i >= 0) p.lse[rowoff] = lse2 * LN2;
-        const uint32_t sO = smem_u32(smem + OFF_Q);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float x[8];
+        for (int e = 0; e < 64; ++e) acc[e] *= w2;
+        if (w1 != 0.f) {  // add the first pass's output with its log-sum-exp weight
+            if (SPLIT) {
+                const float4 *src = reinterpret_cast<const float4 *>(p.o_prev_f32 + rowoff * 64);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = acc[8 * j + e] * w2;
-            if (w1 != 0.f) {
-                const uint32_t pw[4] = {prev[j].x, prev[j].y, prev[j].z, prev[j].w};
+                for (int j = 0; j < 16; ++j) {
+                    const float4 u = src[j];
+                    acc[4 * j] += w1 * u.x;
+                    acc[4 * j + 1] += w1 * u.y;
+                    acc[4 * j + 2] += w1 * u.z;
+                    acc[4 * j + 3] += w1 * u.w;
+                }
+            } else {
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * 64);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[2 * e] += w1 * __uint_as_float(pw[e] << 16);
-                    x[2 * e + 1] += w1 * __uint_as_float(pw[e] & 0xFFFF0000u);
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 u = src[j];
+                    const uint32_t pw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[8 * j + 2 * e] += w1 * bf16_lo(pw[e]);
+                        acc[8 * j + 2 * e + 1] += w1 * bf16_hi(pw[e]);
+                    }
                 }
             }
-            st_shared_v4(sO + sw128_off(row, j), pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                         pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (row == 0 && *abort == 0) {
-            store_tile(p.o, part.qframe, p.g, part.o, w.tile, bh, smem + OFF_Q);
-            bulk_commit();
-            bulk_wait_all();
+        if (SPLIT) {
+            // fp32 output: row by row (64 floats = 256 bytes per row)
+            if (i >= 0 && *abort == 0) {
+                float4 *dst = reinterpret_cast<float4 *>(p.o_f32 + rowoff * 64);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            }
+        } else {
+            const uint32_t sO = smem_u32(smem + OFF_Q);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                st_shared_v4(sO + sw128_off(row, j), pack_bf16(acc[8 * j], acc[8 * j + 1]),
+                             pack_bf16(acc[8 * j + 2], acc[8 * j + 3]),
+                             pack_bf16(acc[8 * j + 4], acc[8 * j + 5]),
+                             pack_bf16(acc[8 * j + 6], acc[8 * j + 7]));
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (row == 0 && *abort == 0) {
+                store_tile(p.o, part.qframe, p.g, part.o, w.tile, bh, smem + OFF_Q);
+                bulk_commit();
+                bulk_wait_all();
+            }
         }
     }
     tc_fence_before();
@@ -289,20 +340,26 @@ __global__ void __launch_bounds__(THREADS, 2) fwd_kernel(const __grid_constant__
     }
 }
 
-}  // namespace
-
-cudaError_t launch_fwd(const FwdParams &p, cudaStream_t s)
+template <bool SPLIT>
+cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t s)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(fwd_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Plan<SPLIT>::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (p.nitems == 0) return cudaSuccess;
-    fwd_kernel<<<dim3(static_cast<unsigned>(p.nitems) * p.batch), THREADS, SMEM_BYTES, s>>>(p);
+    fwd_kernel<SPLIT><<<dim3(static_cast<unsigned>(p.nitems) * p.batch), THREADS, Plan<SPLIT>::SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s)
+{
+    return split ? launch_fwd_t<true>(p, s) : launch_fwd_t<false>(p, s);
 }
 
 }  // namespace st

@@ -18,6 +18,7 @@ struct FrameMaps {
 
 struct FwdParams {
     FrameMaps q, k, v, o;        // o.sum unused
+    FrameMaps ql, kl;            // split precision (fp32 I/O): low bf16 parts of Q and K
     const Part *parts;
     const WorkItem *items;
     int32_t nitems, batch, heads;
@@ -25,6 +26,8 @@ struct FwdParams {
     float scale_log2;            // log2(e) / sqrt(d)
     float *lse;                  // [B*H, n]
     const uint16_t *o_prev;      // merge pass: the output (bf16) written by the first pass
+    float *o_f32;                // fp32 I/O: output written row by row instead of through TMA
+    const float *o_prev_f32;     // fp32 I/O merge pass: the first pass's output
     int32_t *err;                // device error word
 };
 
@@ -42,11 +45,15 @@ struct BwdParams {
     float *dq_acc;               // [B*H, n, 64] fp32, zeroed before the main kernel
     const uint16_t *dk_prev;     // merge pass: dK, dV written by the first pass (bf16)
     const uint16_t *dv_prev;
+    float *dk_f32, *dv_f32;      // fp32 I/O: outputs written row by row
+    const float *dk_prev_f32, *dv_prev_f32;
     int32_t *err;
 };
 
 struct PreParams {
     const uint16_t *o, *dout;    // bf16 [B*H, n, 64]
+    const float *o_f32, *dout_f32;  // fp32 I/O instead of o, dout
+    float *dk_f32, *dv_f32;         // fp32 I/O instead of dk, dv
     float *delta;                // [B*H, n]
     float *dq_acc;               // [B*H, n, 64] zeroed here
     uint16_t *dk, *dv;           // zero-filled for heads flagged in zero_fill
@@ -58,12 +65,21 @@ struct PreParams {
 struct ConvParams {
     const float *dq_acc;
     uint16_t *dq;
+    float *dq_f32;               // fp32 I/O: plain copy instead of rounding to bf16
     int64_t elems;
 };
 
-cudaError_t launch_fwd(const FwdParams &p, cudaStream_t s);
-cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s);
-cudaError_t launch_bwd_pre(const PreParams &p, cudaStream_t s);
-cudaError_t launch_dq_convert(const ConvParams &p, cudaStream_t s);
+// fp32 -> bf16 hi (round to nearest even) and, if lo != nullptr, lo = bf16(x - hi)
+struct SplitParams {
+    const float *src;
+    uint16_t *hi, *lo;
+    int64_t elems;
+};
+
+cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s);
+cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
+cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s);
+cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s);
+cudaError_t launch_split(const SplitParams &p, cudaStream_t s);
 
 }  // namespace st

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from parity import check_grads, cuda_inputs, problem_of, rel_l2, sample_rows, to64
-from test_fwd_gpu import SMALL
+from test_fwd_gpu import FP32, SMALL
 from workloads import WORKLOADS
 
 pytestmark = pytest.mark.gpu
@@ -46,6 +46,15 @@ def test_bwd_small_all_elements(w):
 
 
 BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
+
+
+@pytest.mark.parametrize("w", FP32, ids=lambda w: w.name)
+def test_bwd_fp32_all_elements(w):
+    (qd, kd, vd, dod), (q, k, v, do) = cuda_inputs(w)
+    _, _, _, dq, dk, dv = run(w, qd, kd, vd, dod)
+    assert dq.dtype == dk.dtype == dv.dtype == torch.float32
+    ref = problem_of(w).bwd(to64(q), to64(k), to64(v), to64(do))
+    check_grads((to64(dq), to64(dk), to64(dv)), ref, w.name)
 
 
 def sample_keys(w, count, seed=1):

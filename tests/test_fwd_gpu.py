@@ -56,6 +56,22 @@ def test_fwd_small_all_elements(w):
 
 BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
 
+# fp32 I/O: the n = 256 fp32 workload plus fixed and merged variants, every element compared
+FP32 = [WORKLOADS["strided_n256_l16_fp32"],
+        Workload("f32_fixed_n512_l128_c32", FIXED, ALTERNATING, 512, 128, 32, 1, 4, dtype="fp32"),
+        Workload("f32_s_merged_n768_l24", STRIDED, MERGED, 768, 24, 0, 1, 2, dtype="fp32"),
+        Workload("f32_f_merged_n512_l128_c32", FIXED, MERGED, 512, 128, 32, 1, 2, dtype="fp32")]
+
+
+@pytest.mark.parametrize("w", FP32, ids=lambda w: w.name)
+def test_fwd_fp32_all_elements(w):
+    (qd, kd, vd, _), (q, k, v, _) = cuda_inputs(w)
+    assert qd.dtype == torch.float32
+    _, o, lse = run_fwd(w, qd, kd, vd)
+    assert o.dtype == torch.float32
+    o_ref, lse_ref = problem_of(w).fwd(to64(q), to64(k), to64(v))
+    check_o_lse(to64(o), lse.cpu().numpy(), o_ref, lse_ref, w.name)
+
 
 @pytest.mark.parametrize("w", BIG, ids=lambda w: w.name)
 def test_fwd_full_size_sampled_rows(w):
