@@ -200,6 +200,26 @@ ST_API st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void 
                                       size_t workspace_bytes, const st_desc_t *desc,
                                       st_stream_t stream);
 
+/* Backward pass for callers that cannot allocate device memory (no counterpart in the paper:
+ * this is a deployment convenience).  A plug-in inside a host application that owns every device
+ * allocation, or code that must not pay cudaMalloc's implicit synchronisation, can call this
+ * instead of st_attn_bwd: same arguments and results, but no workspace argument -- the scratch
+ * (fp32 dQ accumulator and D_i) lives in a fixed array of ST_NOALLOC_SCRATCH_BYTES that is part of
+ * the library's device image, held on every GPU that loads the library until the process exits.
+ * Nothing is allocated (no cudaMalloc, cudaFree or allocating library call).
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - Problems whose st_attn_bwd_workspace_bytes exceeds ST_NOALLOC_SCRATCH_BYTES are rejected
+ *     with ST_ERR_WORKSPACE before anything is enqueued (with bf16 I/O that is batch * heads * n
+ *     above about 129,000 rows).
+ *   - All calls on a device share the array; each call re-initialises what it reads, but calls
+ *     whose work overlaps on the GPU (other streams, other threads) race on it. */
+#define ST_NOALLOC_SCRATCH_BYTES (32u << 20)
+ST_API st_status_t st_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                                       const float *lse, const void *dO,
+                                       const st_layout_t *layout, void *dq, void *dk, void *dv,
+                                       const st_desc_t *desc, st_stream_t stream);
+
 /* Static description of a status code. */
 ST_API const char *st_status_string(st_status_t status);
 
