@@ -13,8 +13,10 @@
 //   warp 1      MMA issuer: S = Q K^T and dP = dO V^T (TMEM, 128 x 128 fp32 each), then after
 //               the softmax warps wrote P and dS (bf16, SMEM): dV += P^T dO, dK += dS^T Q
 //               (TMEM 128 x 64 each, resident for the whole item) and dQ = dS K (TMEM 128 x 64)
-//   warps 2..5  one query row per thread: interval mask, P, dS; drain dQ with atomics; at the
-//               end one key row per thread: dK, dV to bf16 and a TMA store.
+//   warps 2..9  two warpgroups, one query row per thread, warpgroup h owning score columns
+//               64h..64h+63 (no row reduction is needed here: P comes from the saved lse):
+//               interval mask, P, dS; drain dQ columns 32h.. with atomics; at the end one key
+//               row per thread: dK, dV columns 32h.. to bf16 and a TMA store.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
 #include "tiles.cuh"
 
@@ -31,7 +33,7 @@ constexpr uint32_t OFF_P = OFF_DO + NST * TB;      // 2 halves; dK/dV staging at
 constexpr uint32_t OFF_DS = OFF_P + 2 * TB;        // 2 halves
 constexpr uint32_t OFF_BAR = OFF_DS + 2 * TB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 320, COL_DQ = 384;
 
@@ -62,9 +64,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->p_full, 256);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 128);
+        mbar_init(&bars->dq_empty, 256);
         for (int s = 0; s < NST; ++s) {
             mbar_init(&bars->qdo_full[s], 1);
             mbar_init(&bars->qdo_empty[s], 1);
@@ -160,14 +162,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             }
         }
     } else {
-        // ---------------- softmax / dS / dQ drain / epilogue (warps 2..5) ----------------
+        // ------- P, dS, dQ drain, epilogue (warps 2..9: warpgroup h owns columns 64h..64h+63) -------
+        const int h = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
+        const int wg_tid = threadIdx.x - 64 - 128 * h;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-        const uint32_t tS = tbase + COL_S + lane_off, tDP = tbase + COL_DP + lane_off;
-        const uint32_t tDQ = tbase + COL_DQ + lane_off;
-        const uint32_t sP = smem_u32(smem + OFF_P), sDS = smem_u32(smem + OFF_DS);
-        const float sc = p.scale_log2;
+        const uint32_t tS = tbase + COL_S + lane_off + 64 * h, tDP = tbase + COL_DP + lane_off + 64 * h;
+        const uint32_t tDQ = tbase + COL_DQ + lane_off + 32 * h;
+        const uint32_t sPh = smem_u32(smem + OFF_P) + h * TB, sDSh = smem_u32(smem + OFF_DS) + h * TB;
+        const float sc = p.scale_log2, dsc = p.ds_scale;
         const size_t head_base = static_cast<size_t>(bh) * p.g.n;
         bool ok = run;
         uint32_t sv[32], dv[32];
@@ -175,93 +179,93 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             const int32_t qt = w.begin + j;
             int32_t lo_abs, hi_abs;
             const int32_t i = row_interval(p.g, part, qt, row, lo_abs, hi_abs);
-            float lse2 = 0.f, Di = 0.f;
+            float nlse = 0.f, nD = 0.f;  // -lse (log2 units) and -D_i / sqrt(d) of this row
             if (i >= 0) {
-                lse2 = p.lse[head_base + i] * LOG2E;
-                Di = p.delta[head_base + i];
+                const float lse = p.lse[head_base + i];
+                // a row with no allowed key (lse = -inf) has every entry masked to -inf below;
+                // keep its base finite so that -inf + base stays -inf instead of NaN
+                nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
+                nD = -p.delta[head_base + i] * dsc;
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, p.err))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int32_t lo = lo_abs - kt * TILE, hi = hi_abs - kt * TILE;
-            const bool full = (lo <= 0) && (hi >= TILE - 1);
+            const int32_t base = kt * TILE + 64 * h;
+            const int32_t lo = lo_abs - base, hi = hi_abs - base;   // allowed columns of this half
+            const bool full = (lo <= 0) && (hi >= 63);
+            const uint32_t span = static_cast<uint32_t>(hi - lo);
+            const bool none = hi < lo;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 tmem_ld32(tS + ch * 32, sv);
                 tmem_ld32(tDP + ch * 32, dv);
                 tmem_wait_ld();
-                uint32_t pk[16], dk[16];
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const bool keep = !none && static_cast<uint32_t>(ch * 32 + e - lo) <= span;
+                        sv[e] = keep ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int c0 = ch * 32 + 2 * e, c1 = c0 + 1;
-                    const bool k0 = full || (c0 >= lo && c0 <= hi);
-                    const bool k1 = full || (c1 >= lo && c1 <= hi);
-                    const float p0 = k0 ? ex2(__uint_as_float(sv[2 * e]) * sc - lse2) : 0.f;
-                    const float p1 = k1 ? ex2(__uint_as_float(sv[2 * e + 1]) * sc - lse2) : 0.f;
-                    const float d0 = p0 * (__uint_as_float(dv[2 * e]) - Di) * p.ds_scale;
-                    const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - Di) * p.ds_scale;
-                    pk[e] = pack_bf16(p0, p1);
-                    dk[e] = pack_bf16(d0, d1);
+                    // P = exp2(S log2e / sqrt(d) - lse log2e);  dS = P (dP - D) / sqrt(d)
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sc, nlse));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sc, nlse));
+                    const float d0 = p0 * fmaf(__uint_as_float(dv[2 * e]), dsc, nD);
+                    const float d1 = p1 * fmaf(__uint_as_float(dv[2 * e + 1]), dsc, nD);
+                    sv[e] = pack_bf16(p0, p1);
+                    dv[e] = pack_bf16(d0, d1);
                 }
-                const uint32_t hp = sP + (ch >> 1) * TB, hd = sDS + (ch >> 1) * TB;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t off = sw128_off(row, (ch & 1) * 4 + q);
-                    st_shared_v4(hp + off, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                    st_shared_v4(hd + off, dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+                    const uint32_t off = sw128_off(row, ch * 4 + q);
+                    st_shared_v4(sPh + off, sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
+                    st_shared_v4(sDSh + off, dv[4 * q], dv[4 * q + 1], dv[4 * q + 2], dv[4 * q + 3]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars->p_full);
-            // drain dQ of this (query tile, key tile) pair into the fp32 accumulator
+            // drain dQ columns 32h .. 32h+31 of this (query tile, key tile) pair
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, j & 1, abort, p.err))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tmem_ld32(tDQ + h * 32, sv);
-                tmem_wait_ld();
-                if (i >= 0) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.dq_acc + (head_base + i) * 64 + h * 32);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        atomicAdd(dst + e, make_float4(__uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]),
-                                                       __uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3])));
-                }
-            }
+            tmem_ld32(tDQ, sv);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
+            if (i >= 0) {
+                float4 *dst = reinterpret_cast<float4 *>(p.dq_acc + (head_base + i) * 64 + 32 * h);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    atomicAdd(dst + e, make_float4(__uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]),
+                                                   __uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3])));
+            }
         }
-        // ---------------- dK, dV epilogue: one key row per thread ----------------
+        // ------- dK, dV epilogue: one key row per thread, warpgroup h writes columns 32h.. -------
         if (ok) {
             const int32_t pos = frame_pos(p.g, part.kframe, part.o, kt, row);
-            const uint32_t sKs = smem_u32(smem + OFF_P), sVs = smem_u32(smem + OFF_P + TB);
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const uint32_t tacc = tbase + (which == 0 ? COL_DK : COL_DV) + lane_off;
-                const uint16_t *prev = which == 0 ? p.dk_prev : p.dv_prev;
-                const uint32_t dst = which == 0 ? sKs : sVs;
-                float acc[64];
+                const uint32_t tacc = tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + 32 * h;
+                float acc[32];
+                tmem_ld32(tacc, sv);
+                tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    tmem_ld32(tacc + h * 32, sv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) acc[h * 32 + e] = __uint_as_float(sv[e]);
-                }
+                for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(sv[e]);
                 if (F32) {
                     if (pos >= 0 && *abort == 0) {
                         const float *pf = which == 0 ? p.dk_prev_f32 : p.dv_prev_f32;
-                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64;
+                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64 + 32 * h;
                         if (part.merge) {
-                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64);
+                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64 + 32 * h);
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) {
+                            for (int q = 0; q < 8; ++q) {
                                 const float4 u = src[q];
                                 acc[4 * q] += u.x;
                                 acc[4 * q + 1] += u.y;
@@ -271,15 +275,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                         }
                         float4 *d4 = reinterpret_cast<float4 *>(of);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q)
+                        for (int q = 0; q < 8; ++q)
                             d4[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
                     }
                     continue;
                 }
                 if (part.merge && pos >= 0) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64);
+                    const uint16_t *prev = which == 0 ? p.dk_prev : p.dv_prev;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64 + 32 * h);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < 4; ++q) {
                         const uint4 u = src[q];
                         const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -289,17 +294,18 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                         }
                     }
                 }
+                const uint32_t dst = smem_u32(smem + OFF_P) + which * TB;  // staging: dK, dV tiles
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    st_shared_v4(dst + sw128_off(row, q), pack_bf16(acc[8 * q], acc[8 * q + 1]),
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(dst + sw128_off(row, 4 * h + q), pack_bf16(acc[8 * q], acc[8 * q + 1]),
                                  pack_bf16(acc[8 * q + 2], acc[8 * q + 3]),
                                  pack_bf16(acc[8 * q + 4], acc[8 * q + 5]),
                                  pack_bf16(acc[8 * q + 6], acc[8 * q + 7]));
             }
             fence_proxy_async_smem();
         }
-        named_bar_sync(1, 128);
-        if (!F32 && row == 0 && ok && *abort == 0) {
+        named_bar_sync(1, 256);
+        if (!F32 && h == 0 && wg_tid == 0 && ok && *abort == 0) {
             store_tile(p.dk, part.kframe, p.g, part.o, kt, bh, smem + OFF_P);
             store_tile(p.dv, part.kframe, p.g, part.o, kt, bh, smem + OFF_P + TB);
             bulk_commit();
