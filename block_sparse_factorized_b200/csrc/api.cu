@@ -64,6 +64,30 @@ bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH
     return true;
 }
 
+// fp32 [BH, n, 64] maps with 32-column (128-byte), 32-row boxes: the dQ accumulator as the
+// reduce target of one warp's slice.
+bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col)
+{
+    memset(&m, 0, sizeof(m));
+    const cuuint64_t row = 64 * 4, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
+    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    {
+        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[2] = {row, n * row};
+        const cuuint32_t box[3] = {32, 32, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box)) return false;
+    }
+    if (col) {
+        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[3] = {l * row, row, n * row};
+        const cuuint32_t rows = static_cast<cuuint32_t>(g.Rt < 32 ? g.Rt : 32);
+        const cuuint32_t slots = static_cast<cuuint32_t>(g.Rt < 32 ? 32 / g.Rt : 1);
+        const cuuint32_t box[4] = {32, rows, slots, 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box)) return false;
+    }
+    return true;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Frames {
@@ -279,6 +303,7 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
         p.dk_prev_f32 = static_cast<const float *>(dk);
         p.dv_prev_f32 = static_cast<const float *>(dv);
     }
+    if (!make_maps_f32(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol)) return ST_ERR_CUDA;
     if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false) ||
         !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum))
         return ST_ERR_CUDA;

@@ -31,14 +31,15 @@ constexpr uint32_t OFF_Q = OFF_V + TB;             // NST tiles
 constexpr uint32_t OFF_DO = OFF_Q + NST * TB;      // NST tiles
 constexpr uint32_t OFF_P = OFF_DO + NST * TB;      // 2 halves; dK/dV staging at the end
 constexpr uint32_t OFF_DS = OFF_P + 2 * TB;        // 2 halves
-constexpr uint32_t OFF_BAR = OFF_DS + 2 * TB;
+constexpr uint32_t OFF_DQ = OFF_DS + 2 * TB;       // dQ staging: 2 x (128 rows x 32 fp32)
+constexpr uint32_t OFF_BAR = OFF_DQ + 2 * TB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 320, COL_DQ = 384;
 
 struct Bars {
-    uint64_t kv_full, s_full, p_full, dq_full, dq_empty;
+    uint64_t kv_full, s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
     uint64_t qdo_full[NST], qdo_empty[NST];
     uint32_t tmem_base;
     int32_t abort;
@@ -64,7 +65,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 256);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_ready, 256);
+        mbar_init(&bars->ds_ready, 256);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 256);
         for (int s = 0; s < NST; ++s) {
@@ -119,46 +122,64 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             constexpr uint32_t id_kt = idesc_bf16(128, 64, false, true);    // dQ
             const uint32_t sK = smem_u32(smem + OFF_K), sV = smem_u32(smem + OFF_V);
             const uint32_t sP = smem_u32(smem + OFF_P), sDS = smem_u32(smem + OFF_DS);
-            if (mbar_wait(&bars->kv_full, 0, abort, p.err)) {
-                for (int j = 0; j < nq; ++j) {
-                    const int s = j % NST;
-                    if (!mbar_wait(&bars->qdo_full[s], (j / NST) & 1, abort, p.err)) break;
+            // Per query tile j the tensor core runs, in order:
+            //   dV += P_j^T dO_j | S_{j+1} | dK += dS_j^T Q_j, dQ_j = dS_j K | dP_{j+1}
+            // so that it computes dV_j and S_{j+1} while the softmax warps build dS_j, and dK_j,
+            // dQ_j, dP_{j+1} while they drain dQ_j and build P_{j+1}.
+            auto issue_s = [&](uint32_t sQ) {  // S = Q K^T (both K-major over d)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ss(tbase + COL_S, desc_sw128(sQ + 32 * k, 16, 1024),
+                                desc_sw128(sK + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full);
+            };
+            auto issue_dp = [&](uint32_t sDO) {  // dP = dO V^T
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ss(tbase + COL_DP, desc_sw128(sDO + 32 * k, 16, 1024),
+                                desc_sw128(sV + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
+                mma_commit(&bars->dp_full);
+            };
+            bool go = mbar_wait(&bars->kv_full, 0, abort, p.err) &&
+                      mbar_wait(&bars->qdo_full[0], 0, abort, p.err);
+            if (go) {
+                tc_fence_after();
+                issue_s(smem_u32(smem + OFF_Q));
+                issue_dp(smem_u32(smem + OFF_DO));
+            }
+            for (int j = 0; go && j < nq; ++j) {
+                const int s = j % NST, s1 = (j + 1) % NST;
+                const uint32_t sQ = smem_u32(smem + OFF_Q + s * TB);
+                const uint32_t sDO = smem_u32(smem + OFF_DO + s * TB);
+                const bool next = j + 1 < nq;
+                if (!mbar_wait(&bars->p_ready, j & 1, abort, p.err)) break;
+                tc_fence_after();
+                // dV += P^T dO: A = P^T MN-major (two 64-key atoms 16 KB apart), B = dO
+                // MN-major; 16 queries (2048 bytes) per step
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + k * 2048, TB, 1024),
+                                desc_sw128(sDO + k * 2048, TB, 1024), id_tt, (j > 0 || k > 0) ? 1u : 0u);
+                if (next) {  // S of the next query tile: the softmax warps are done reading S_j
+                    if (!mbar_wait(&bars->qdo_full[s1], ((j + 1) / NST) & 1, abort, p.err)) break;
                     tc_fence_after();
-                    const uint32_t sQ = smem_u32(smem + OFF_Q + s * TB);
-                    const uint32_t sDO = smem_u32(smem + OFF_DO + s * TB);
-                    // S = Q K^T, dP = dO V^T (all K-major over d)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ss(tbase + COL_S, desc_sw128(sQ + 32 * k, 16, 1024),
-                                    desc_sw128(sK + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ss(tbase + COL_DP, desc_sw128(sDO + 32 * k, 16, 1024),
-                                    desc_sw128(sV + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full);
-                    if (!mbar_wait(&bars->p_full, j & 1, abort, p.err)) break;
-                    if (j > 0 && !mbar_wait(&bars->dq_empty, (j - 1) & 1, abort, p.err)) break;
-                    tc_fence_after();
-                    // dV += P^T dO, dK += dS^T Q: A = P^T / dS^T MN-major (two 64-key atoms,
-                    // 16 KB apart), B = dO / Q MN-major; 16 queries (2048 bytes) per step
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + k * 2048, TB, 1024),
-                                    desc_sw128(sDO + k * 2048, TB, 1024), id_tt,
-                                    (j > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + k * 2048, TB, 1024),
-                                    desc_sw128(sQ + k * 2048, TB, 1024), id_tt,
-                                    (j > 0 || k > 0) ? 1u : 0u);
-                    // dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (k >> 2) * TB + (k & 3) * 32, 16, 1024),
-                                    desc_sw128(sK + k * 2048, TB, 1024), id_kt, k > 0 ? 1u : 0u);
-                    mma_commit(&bars->dq_full);
-                    mma_commit(&bars->qdo_empty[s]);
+                    issue_s(smem_u32(smem + OFF_Q + s1 * TB));
                 }
+                if (!mbar_wait(&bars->ds_ready, j & 1, abort, p.err)) break;
+                if (j > 0 && !mbar_wait(&bars->dq_empty, (j - 1) & 1, abort, p.err)) break;
+                tc_fence_after();
+                // dK += dS^T Q (as dV), dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + k * 2048, TB, 1024),
+                                desc_sw128(sQ + k * 2048, TB, 1024), id_tt, (j > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (k >> 2) * TB + (k & 3) * 32, 16, 1024),
+                                desc_sw128(sK + k * 2048, TB, 1024), id_kt, k > 0 ? 1u : 0u);
+                mma_commit(&bars->dq_full);
+                mma_commit(&bars->qdo_empty[s]);
+                if (next) issue_dp(smem_u32(smem + OFF_DO + s1 * TB));  // dP_j already consumed
             }
         }
     } else {
@@ -171,15 +192,28 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         const uint32_t tS = tbase + COL_S + lane_off + 64 * h, tDP = tbase + COL_DP + lane_off + 64 * h;
         const uint32_t tDQ = tbase + COL_DQ + lane_off + 32 * h;
         const uint32_t sPh = smem_u32(smem + OFF_P) + h * TB, sDSh = smem_u32(smem + OFF_DS) + h * TB;
+        const uint32_t sDQw = smem_u32(smem + OFF_DQ) + h * TB + q4 * 4096;  // this warp's staging
         const float sc = p.scale_log2, dsc = p.ds_scale;
         const size_t head_base = static_cast<size_t>(bh) * p.g.n;
         bool ok = run;
         uint32_t sv[32], dv[32];
-        for (int j = 0; ok && j < nq; ++j) {
-            const int32_t qt = w.begin + j;
+        float pr[64];                  // P of this row's 64 columns, kept from P_j to dS_j
+        float nlse = 0.f, nD = 0.f;    // -lse (log2 units) and -D_i / sqrt(d) of the row
+        int32_t lo = 1, hi = 0;        // allowed columns of this half, relative to the half
+        // Order per query tile: P_0; then for each j: dS_j, P_{j+1}, drain dQ_j.  Building P_{j+1}
+        // while the tensor core computes dK_j and dQ_j hides their latency.  Buffer safety comes
+        // from commit order: S_{j+1} is issued after dV_j (so s_full(j+1) means P_j was read) and
+        // dP_{j+1} after dK_j, dQ_j (so dp_full(j+1) means dS_j was read).
+        auto wait_all = [&](uint64_t *bar, int parity) {
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.err));
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        auto p_phase = [&](int j) {    // P_j = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
             int32_t lo_abs, hi_abs;
-            const int32_t i = row_interval(p.g, part, qt, row, lo_abs, hi_abs);
-            float nlse = 0.f, nD = 0.f;  // -lse (log2 units) and -D_i / sqrt(d) of this row
+            const int32_t i = row_interval(p.g, part, w.begin + j, row, lo_abs, hi_abs);
+            nlse = 0.f;
+            nD = 0.f;
             if (i >= 0) {
                 const float lse = p.lse[head_base + i];
                 // a row with no allowed key (lse = -inf) has every entry masked to -inf below;
@@ -187,20 +221,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
                 nD = -p.delta[head_base + i] * dsc;
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, p.err))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
             const int32_t base = kt * TILE + 64 * h;
-            const int32_t lo = lo_abs - base, hi = hi_abs - base;   // allowed columns of this half
+            lo = lo_abs - base;
+            hi = hi_abs - base;
+            if (!wait_all(&bars->s_full, j & 1)) return;
             const bool full = (lo <= 0) && (hi >= 63);
             const uint32_t span = static_cast<uint32_t>(hi - lo);
             const bool none = hi < lo;
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 tmem_ld32(tS + ch * 32, sv);
-                tmem_ld32(tDP + ch * 32, dv);
                 tmem_wait_ld();
                 if (!full) {
 #pragma unroll
@@ -210,43 +240,68 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    // P = exp2(S log2e / sqrt(d) - lse log2e);  dS = P (dP - D) / sqrt(d)
-                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sc, nlse));
-                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sc, nlse));
-                    const float d0 = p0 * fmaf(__uint_as_float(dv[2 * e]), dsc, nD);
-                    const float d1 = p1 * fmaf(__uint_as_float(dv[2 * e + 1]), dsc, nD);
-                    sv[e] = pack_bf16(p0, p1);
-                    dv[e] = pack_bf16(d0, d1);
-                }
+                for (int e = 0; e < 32; ++e) pr[ch * 32 + e] = ex2(fmaf(__uint_as_float(sv[e]), sc, nlse));
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(sPh + sw128_off(row, ch * 4 + q),
+                                 pack_bf16(pr[ch * 32 + 8 * q], pr[ch * 32 + 8 * q + 1]),
+                                 pack_bf16(pr[ch * 32 + 8 * q + 2], pr[ch * 32 + 8 * q + 3]),
+                                 pack_bf16(pr[ch * 32 + 8 * q + 4], pr[ch * 32 + 8 * q + 5]),
+                                 pack_bf16(pr[ch * 32 + 8 * q + 6], pr[ch * 32 + 8 * q + 7]));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->p_ready);
+        };
+        auto ds_phase = [&](int j) {   // dS_j = P (dP - D) / sqrt(d) -> SMEM
+            if (!wait_all(&bars->dp_full, j & 1)) return;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                tmem_ld32(tDP + ch * 32, dv);
+                tmem_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t off = sw128_off(row, ch * 4 + q);
-                    st_shared_v4(sPh + off, sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
-                    st_shared_v4(sDSh + off, dv[4 * q], dv[4 * q + 1], dv[4 * q + 2], dv[4 * q + 3]);
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 8 * q + 2 * e;
+                        pk[e] = pack_bf16(pr[ch * 32 + c] * fmaf(__uint_as_float(dv[c]), dsc, nD),
+                                          pr[ch * 32 + c + 1] * fmaf(__uint_as_float(dv[c + 1]), dsc, nD));
+                    }
+                    st_shared_v4(sDSh + sw128_off(row, ch * 4 + q), pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
-            // drain dQ columns 32h .. 32h+31 of this (query tile, key tile) pair
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, j & 1, abort, p.err))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+            mbar_arrive(&bars->ds_ready);
+        };
+        auto drain = [&](int j) {      // dQ_j columns 32h.. : TMEM -> SMEM -> TMA reduce-add
+            if (!wait_all(&bars->dq_full, j & 1)) return;
             tmem_ld32(tDQ, sv);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
-            if (i >= 0) {
-                float4 *dst = reinterpret_cast<float4 *>(p.dq_acc + (head_base + i) * 64 + 32 * h);
+            // per-warp staging (32 rows x 128 bytes, 1024-byte aligned): no cross-warp barrier
+            if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce has read it
+            __syncwarp();
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    atomicAdd(dst + e, make_float4(__uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]),
-                                                   __uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3])));
+            for (int q = 0; q < 8; ++q)
+                st_shared_v4(sDQw + sw128_off(lane, q), sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                reduce_warp_f32(p.dq_red, part.qframe, p.g, w.begin + j, bh, h, q4,
+                                smem + OFF_DQ + h * TB + q4 * 4096);
+                bulk_commit();
             }
+        };
+        if (ok) p_phase(0);
+        for (int j = 0; ok && j < nq; ++j) {
+            ds_phase(j);
+            if (ok && j + 1 < nq) p_phase(j + 1);
+            if (ok) drain(j);
         }
+        if (lane == 0) bulk_wait_all();  // every dQ reduce of this warp has landed
         // ------- dK, dV epilogue: one key row per thread, warpgroup h writes columns 32h.. -------
         if (ok) {
             const int32_t pos = frame_pos(p.g, part.kframe, part.o, kt, row);

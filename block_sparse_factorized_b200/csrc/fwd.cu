@@ -54,7 +54,7 @@ struct Plan {
 
 struct Bars {
     uint64_t q_full, s_full, o_done;
-    uint64_t p_full[2];
+    uint64_t p_full[2], pv_done[2];
     uint64_t kv_full[NST], kv_empty[NST];
     uint32_t tmem_base;
     int32_t abort;
@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->p_full[0], 128);
         mbar_init(&bars->p_full[1], 128);
+        mbar_init(&bars->pv_done[0], 1);
+        mbar_init(&bars->pv_done[1], 1);
         for (int s = 0; s < NST; ++s) {
             mbar_init(&bars->kv_full[s], 1);
             mbar_init(&bars->kv_empty[s], 1);
@@ -156,49 +158,60 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idO = idesc_bf16(128, 64, false, true);
             const uint32_t sQ = smem_u32(smem + L::OFF_Q), sP = smem_u32(smem + L::OFF_P);
-            if (mbar_wait(&bars->q_full, 0, abort, p.err)) {
-                for (int it = 0; it < nkt; ++it) {
-                    const int s = it % NST;
-                    if (!mbar_wait(&bars->kv_full[s], (it / NST) & 1, abort, p.err)) break;
-                    tc_fence_after();
-                    const uint32_t sK = smem_u32(smem + L::OFF_STAGE + s * L::STAGE);
-                    const uint32_t sV = sK + TB;
-                    // S = Q K^T: both operands K-major, 16 elements (32 bytes) of d per step.
-                    // Split precision adds Q_hi K_lo^T + Q_lo K_hi^T into the same accumulator.
+            // S = Q K^T: both operands K-major, 16 elements (32 bytes) of d per step.  Split
+            // precision adds Q_hi K_lo^T + Q_lo K_hi^T into the same accumulator.
+            auto issue_s = [&](int it) {
+                const uint32_t sK = smem_u32(smem + L::OFF_STAGE + (it % NST) * L::STAGE);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
+                                desc_sw128(sK + 32 * k, 16, 1024), idS, k > 0 ? 1u : 0u);
+                if (SPLIT) {
+                    const uint32_t sQl = smem_u32(smem + L::OFF_QL), sKl = sK + 2 * TB;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
                         mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
-                                    desc_sw128(sK + 32 * k, 16, 1024), idS, k > 0 ? 1u : 0u);
-                    if (SPLIT) {
-                        const uint32_t sQl = smem_u32(smem + L::OFF_QL), sKl = sK + 2 * TB;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
-                                        desc_sw128(sKl + 32 * k, 16, 1024), idS, 1u);
-                            mma_bf16_ss(tS, desc_sw128(sQl + 32 * k, 16, 1024),
-                                        desc_sw128(sK + 32 * k, 16, 1024), idS, 1u);
-                        }
+                                    desc_sw128(sKl + 32 * k, 16, 1024), idS, 1u);
+                        mma_bf16_ss(tS, desc_sw128(sQl + 32 * k, 16, 1024),
+                                    desc_sw128(sK + 32 * k, 16, 1024), idS, 1u);
                     }
-                    mma_commit(&bars->s_full);
-                    // O_h += P_h V_h per key half: P_h K-major (64 keys, 32 bytes per step),
-                    // V_h MN-major (rows 64h.., 16 keys = 2048 bytes per step)
-                    bool fail = false;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (!mbar_wait(&bars->p_full[h], it & 1, abort, p.err)) { fail = true; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16_ss(tbase + 128 + 64 * h,
-                                        desc_sw128(sP + h * TB + k * 32, 16, 1024),
-                                        desc_sw128(sV + h * 8192 + k * 2048, TB, 1024), idO,
-                                        (it > 0 || k > 0) ? 1u : 0u);
-                    }
-                    if (fail) break;
-                    mma_commit(&bars->kv_empty[s]);
                 }
-                mma_commit(&bars->o_done);
+                mma_commit(&bars->s_full);
+            };
+            // O_h += P_h V_h: P_h K-major (64 keys, 32 bytes per step), V_h MN-major (rows 64h..,
+            // 16 keys = 2048 bytes per step)
+            auto issue_pv = [&](int it, int h) {
+                const uint32_t sV = smem_u32(smem + L::OFF_STAGE + (it % NST) * L::STAGE) + TB;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ss(tbase + 128 + 64 * h, desc_sw128(sP + h * TB + k * 32, 16, 1024),
+                                desc_sw128(sV + h * 8192 + k * 2048, TB, 1024), idO,
+                                (it > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bars->pv_done[h]);
+            };
+            // Order per key tile: PV_0(it) | S(it+1) | PV_1(it): the next scores are computed as
+            // soon as both halves have read S(it), while half 1's PV is still pending.
+            bool go = mbar_wait(&bars->q_full, 0, abort, p.err) &&
+                      mbar_wait(&bars->kv_full[0], 0, abort, p.err);
+            if (go) {
+                tc_fence_after();
+                issue_s(0);
             }
+            for (int it = 0; go && it < nkt; ++it) {
+                if (!mbar_wait(&bars->p_full[0], it & 1, abort, p.err)) break;
+                tc_fence_after();
+                issue_pv(it, 0);
+                if (!mbar_wait(&bars->p_full[1], it & 1, abort, p.err)) break;
+                tc_fence_after();
+                if (it + 1 < nkt) {
+                    if (!mbar_wait(&bars->kv_full[(it + 1) % NST], ((it + 1) / NST) & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    issue_s(it + 1);
+                }
+                issue_pv(it, 1);
+                mma_commit(&bars->kv_empty[it % NST]);
+            }
+            if (go) mma_commit(&bars->o_done);
         }
     } else {
         // ---------------- softmax of one key half + epilogue (warps 2..9) ----------------
@@ -253,12 +266,18 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 ps[(c >> 1) & 7] += p0 + p1;
                 v[c >> 1] = pack_bf16(p0, p1);
             }
+            // PV of the previous tile must be done with P_h and O_h before they change
+            if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[h], (it - 1) & 1, abort, p.err))) {
+                ok = false;
+                break;
+            }
+            if (it > 0) tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 st_shared_v4(sPh + sw128_off(row, j), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             if (it > 0 && __any_sync(0xffffffffu, grow)) {
-                // rescale this half's partial O (PV of the previous tile is complete: the S
-                // commit of this tile covers every earlier MMA; PV of this tile waits for p_full)
+                // rescale this half's partial O (complete: pv_done above; PV of this tile waits
+                // for p_full)
                 uint32_t o[32];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {

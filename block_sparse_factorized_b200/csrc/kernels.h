@@ -34,6 +34,8 @@ struct FwdParams {
 struct BwdParams {
     FrameMaps q, k, v, dout;
     FrameMaps dk, dv;            // stores (sum used for compacted keys)
+    FrameMaps dq_red;            // fp32 dQ accumulator in the query frames, box 32 columns wide
+                                 // (reduce-add target; nat and col only)
     const Part *parts;
     const WorkItem *items;
     int32_t nitems, batch, heads;

@@ -125,7 +125,30 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *m, const void *s
         : "memory");
 }
 
+// Element-wise add of a shared-memory tile into global memory (reduction done by the copy engine
+// at L2; elements outside the tensor are skipped).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *m, const void *src, int32_t c0,
+                                                  int32_t c1, int32_t c2)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *m, const void *src, int32_t c0,
+                                                  int32_t c1, int32_t c2, int32_t c3)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+        " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk group has finished reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA store, tensor core).
