@@ -28,11 +28,12 @@ EncodeTiledFn encode_fn()
 }
 
 bool encode(CUtensorMap *m, const void *base, CUtensorMapDataType dt, cuuint32_t rank,
-            const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box)
+            const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     const cuuint32_t es[4] = {1, 1, 1, 1};
     return encode_fn()(m, dt, rank, const_cast<void *>(base), dims, strides, box, es,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -64,8 +65,8 @@ bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH
     return true;
 }
 
-// fp32 [BH, n, 64] maps with 32-column (128-byte), 32-row boxes: the dQ accumulator as the
-// reduce target of one warp's slice.
+// fp32 [BH, n, 64] maps with 16-column (64-byte, 64-byte swizzle), 32-row boxes: the dQ
+// accumulator as the reduce target of one warp's slice.
 bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col)
 {
     memset(&m, 0, sizeof(m));
@@ -74,16 +75,16 @@ bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_
     {
         const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[2] = {row, n * row};
-        const cuuint32_t box[3] = {32, 32, 1};
-        if (!encode(&m.nat, base, dt, 3, dims, str, box)) return false;
+        const cuuint32_t box[3] = {16, 32, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
     }
     if (col) {
         const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[3] = {l * row, row, n * row};
         const cuuint32_t rows = static_cast<cuuint32_t>(g.Rt < 32 ? g.Rt : 32);
         const cuuint32_t slots = static_cast<cuuint32_t>(g.Rt < 32 ? 32 / g.Rt : 1);
-        const cuuint32_t box[4] = {32, rows, slots, 1};
-        if (!encode(&m.col, base, dt, 4, dims, str, box)) return false;
+        const cuuint32_t box[4] = {16, rows, slots, 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
     }
     return true;
 }

@@ -13,10 +13,11 @@
 //   warp 1      MMA issuer: S = Q K^T and dP = dO V^T (TMEM, 128 x 128 fp32 each), then after
 //               the softmax warps wrote P and dS (bf16, SMEM): dV += P^T dO, dK += dS^T Q
 //               (TMEM 128 x 64 each, resident for the whole item) and dQ = dS K (TMEM 128 x 64)
-//   warps 2..9  two warpgroups, one query row per thread, warpgroup h owning score columns
-//               64h..64h+63 (no row reduction is needed here: P comes from the saved lse):
-//               interval mask, P, dS; drain dQ columns 32h.. with atomics; at the end one key
-//               row per thread: dK, dV columns 32h.. to bf16 and a TMA store.
+//   warps 2..17 four warpgroups, one query row per thread, warpgroup g owning score columns
+//               32g..32g+31 (no row reduction is needed here: P comes from the saved lse):
+//               interval mask, P, dS; dQ columns 16g.. staged per warp and added to the fp32
+//               accumulator with a TMA reduce; at the end one key row per thread: dK, dV
+//               columns 16g.. to bf16 and a TMA store.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
 #include "tiles.cuh"
 
@@ -34,7 +35,10 @@ constexpr uint32_t OFF_DS = OFF_P + 2 * TB;        // 2 halves
 constexpr uint32_t OFF_DQ = OFF_DS + 2 * TB;       // dQ staging: 2 x (128 rows x 32 fp32)
 constexpr uint32_t OFF_BAR = OFF_DQ + 2 * TB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
-constexpr int THREADS = 320;
+constexpr int NWG = 4;                             // softmax warpgroups
+constexpr int THREADS = 64 + 128 * NWG;
+constexpr int CW = 128 / NWG;                       // score columns per warpgroup (32)
+constexpr int OW = 64 / NWG;                        // dQ / dK / dV columns per warpgroup (16)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 320, COL_DQ = 384;
 
@@ -66,10 +70,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->dp_full, 1);
-        mbar_init(&bars->p_ready, 256);
-        mbar_init(&bars->ds_ready, 256);
+        mbar_init(&bars->p_ready, 128 * NWG);
+        mbar_init(&bars->ds_ready, 128 * NWG);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 256);
+        mbar_init(&bars->dq_empty, 128 * NWG);
         for (int s = 0; s < NST; ++s) {
             mbar_init(&bars->qdo_full[s], 1);
             mbar_init(&bars->qdo_empty[s], 1);
@@ -183,23 +187,27 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             }
         }
     } else {
-        // ------- P, dS, dQ drain, epilogue (warps 2..9: warpgroup h owns columns 64h..64h+63) -------
-        const int h = (warp - 2) >> 2;
+        // ------- P, dS, dQ drain, epilogue (warps 2..: warpgroup g owns score columns CW g..) -------
+        const int g = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
-        const int wg_tid = threadIdx.x - 64 - 128 * h;
+        const int wg_tid = threadIdx.x - 64 - 128 * g;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-        const uint32_t tS = tbase + COL_S + lane_off + 64 * h, tDP = tbase + COL_DP + lane_off + 64 * h;
-        const uint32_t tDQ = tbase + COL_DQ + lane_off + 32 * h;
-        const uint32_t sPh = smem_u32(smem + OFF_P) + h * TB, sDSh = smem_u32(smem + OFF_DS) + h * TB;
-        const uint32_t sDQw = smem_u32(smem + OFF_DQ) + h * TB + q4 * 4096;  // this warp's staging
+        const uint32_t tS = tbase + COL_S + lane_off + CW * g, tDP = tbase + COL_DP + lane_off + CW * g;
+        const uint32_t tDQ = tbase + COL_DQ + lane_off + OW * g;
+        // P and dS live in two 128 x 64 swizzled halves; this warpgroup's 32 columns are four
+        // 16-byte chunks of half g/2
+        const uint32_t sPg = smem_u32(smem + OFF_P) + (g >> 1) * TB, sDSg = smem_u32(smem + OFF_DS) + (g >> 1) * TB;
+        const uint32_t chunk0 = (g & 1) * 4;
+        const uint32_t warp_slot = (g * 4 + q4) * 2048;     // this warp's dQ staging (32 x 64 B)
+        const uint32_t sDQw = smem_u32(smem + OFF_DQ) + warp_slot;
         const float sc = p.scale_log2, dsc = p.ds_scale;
         const size_t head_base = static_cast<size_t>(bh) * p.g.n;
         bool ok = run;
         uint32_t sv[32], dv[32];
-        float pr[64];                  // P of this row's 64 columns, kept from P_j to dS_j
+        float pr[CW];                  // P of this row's CW columns, kept from P_j to dS_j
         float nlse = 0.f, nD = 0.f;    // -lse (log2 units) and -D_i / sqrt(d) of the row
-        int32_t lo = 1, hi = 0;        // allowed columns of this half, relative to the half
+        int32_t lo = 1, hi = 0;        // allowed columns of this slice, relative to the slice
         // Order per query tile: P_0; then for each j: dS_j, P_{j+1}, drain dQ_j.  Building P_{j+1}
         // while the tensor core computes dK_j and dQ_j hides their latency.  Buffer safety comes
         // from commit order: S_{j+1} is issued after dV_j (so s_full(j+1) means P_j was read) and
@@ -221,77 +229,69 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
                 nD = -p.delta[head_base + i] * dsc;
             }
-            const int32_t base = kt * TILE + 64 * h;
+            const int32_t base = kt * TILE + CW * g;
             lo = lo_abs - base;
             hi = hi_abs - base;
             if (!wait_all(&bars->s_full, j & 1)) return;
-            const bool full = (lo <= 0) && (hi >= 63);
-            const uint32_t span = static_cast<uint32_t>(hi - lo);
-            const bool none = hi < lo;
+            tmem_ld32(tS, sv);
+            tmem_wait_ld();
+            if (!(lo <= 0 && hi >= CW - 1)) {
+                const uint32_t span = static_cast<uint32_t>(hi - lo);
+                const bool none = hi < lo;
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                tmem_ld32(tS + ch * 32, sv);
-                tmem_wait_ld();
-                if (!full) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const bool keep = !none && static_cast<uint32_t>(ch * 32 + e - lo) <= span;
-                        sv[e] = keep ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
-                    }
+                for (int e = 0; e < CW; ++e) {
+                    const bool keep = !none && static_cast<uint32_t>(e - lo) <= span;
+                    sv[e] = keep ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
                 }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) pr[ch * 32 + e] = ex2(fmaf(__uint_as_float(sv[e]), sc, nlse));
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    st_shared_v4(sPh + sw128_off(row, ch * 4 + q),
-                                 pack_bf16(pr[ch * 32 + 8 * q], pr[ch * 32 + 8 * q + 1]),
-                                 pack_bf16(pr[ch * 32 + 8 * q + 2], pr[ch * 32 + 8 * q + 3]),
-                                 pack_bf16(pr[ch * 32 + 8 * q + 4], pr[ch * 32 + 8 * q + 5]),
-                                 pack_bf16(pr[ch * 32 + 8 * q + 6], pr[ch * 32 + 8 * q + 7]));
             }
+#pragma unroll
+            for (int e = 0; e < CW; ++e) pr[e] = ex2(fmaf(__uint_as_float(sv[e]), sc, nlse));
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(sPg + sw128_off(row, chunk0 + q), pack_bf16(pr[8 * q], pr[8 * q + 1]),
+                             pack_bf16(pr[8 * q + 2], pr[8 * q + 3]), pack_bf16(pr[8 * q + 4], pr[8 * q + 5]),
+                             pack_bf16(pr[8 * q + 6], pr[8 * q + 7]));
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars->p_ready);
         };
         auto ds_phase = [&](int j) {   // dS_j = P (dP - D) / sqrt(d) -> SMEM
             if (!wait_all(&bars->dp_full, j & 1)) return;
+            tmem_ld32(tDP, dv);
+            tmem_wait_ld();
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                tmem_ld32(tDP + ch * 32, dv);
-                tmem_wait_ld();
+            for (int q = 0; q < 4; ++q) {
+                uint32_t pk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 8 * q + 2 * e;
-                        pk[e] = pack_bf16(pr[ch * 32 + c] * fmaf(__uint_as_float(dv[c]), dsc, nD),
-                                          pr[ch * 32 + c + 1] * fmaf(__uint_as_float(dv[c + 1]), dsc, nD));
-                    }
-                    st_shared_v4(sDSh + sw128_off(row, ch * 4 + q), pk[0], pk[1], pk[2], pk[3]);
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 8 * q + 2 * e;
+                    pk[e] = pack_bf16(pr[c] * fmaf(__uint_as_float(dv[c]), dsc, nD),
+                                      pr[c + 1] * fmaf(__uint_as_float(dv[c + 1]), dsc, nD));
                 }
+                st_shared_v4(sDSg + sw128_off(row, chunk0 + q), pk[0], pk[1], pk[2], pk[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars->ds_ready);
         };
-        auto drain = [&](int j) {      // dQ_j columns 32h.. : TMEM -> SMEM -> TMA reduce-add
+        auto drain = [&](int j) {      // dQ_j columns OW g.. : TMEM -> SMEM -> TMA reduce-add
             if (!wait_all(&bars->dq_full, j & 1)) return;
-            tmem_ld32(tDQ, sv);
+            uint32_t dq[16];
+            tmem_ld16(tDQ, dq);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
-            // per-warp staging (32 rows x 128 bytes, 1024-byte aligned): no cross-warp barrier
+            // per-warp staging (32 rows x 64 bytes, 64-byte swizzle): no cross-warp barrier
             if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce has read it
             __syncwarp();
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                st_shared_v4(sDQw + sw128_off(lane, q), sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(sDQw + sw64_off(lane, q), dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                reduce_warp_f32(p.dq_red, part.qframe, p.g, w.begin + j, bh, h, q4,
-                                smem + OFF_DQ + h * TB + q4 * 4096);
+                reduce_warp_f32(p.dq_red, part.qframe, p.g, w.begin + j, bh, OW * g, q4,
+                                smem + OFF_DQ + warp_slot);
                 bulk_commit();
             }
         };
@@ -302,25 +302,25 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             if (ok) drain(j);
         }
         if (lane == 0) bulk_wait_all();  // every dQ reduce of this warp has landed
-        // ------- dK, dV epilogue: one key row per thread, warpgroup h writes columns 32h.. -------
+        // ------- dK, dV epilogue: one key row per thread, warpgroup g writes columns OW g.. -------
         if (ok) {
             const int32_t pos = frame_pos(p.g, part.kframe, part.o, kt, row);
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const uint32_t tacc = tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + 32 * h;
-                float acc[32];
-                tmem_ld32(tacc, sv);
+                uint32_t a16[16];
+                tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
                 tmem_wait_ld();
+                float acc[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(sv[e]);
+                for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(a16[e]);
                 if (F32) {
                     if (pos >= 0 && *abort == 0) {
                         const float *pf = which == 0 ? p.dk_prev_f32 : p.dv_prev_f32;
-                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64 + 32 * h;
+                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64 + OW * g;
                         if (part.merge) {
-                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64 + 32 * h);
+                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64 + OW * g);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
+                            for (int q = 0; q < 4; ++q) {
                                 const float4 u = src[q];
                                 acc[4 * q] += u.x;
                                 acc[4 * q + 1] += u.y;
@@ -330,16 +330,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                         }
                         float4 *d4 = reinterpret_cast<float4 *>(of);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
+                        for (int q = 0; q < 4; ++q)
                             d4[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
                     }
                     continue;
                 }
                 if (part.merge && pos >= 0) {
                     const uint16_t *prev = which == 0 ? p.dk_prev : p.dv_prev;
-                    const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64 + 32 * h);
+                    const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64 + OW * g);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 2; ++q) {
                         const uint4 u = src[q];
                         const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -351,16 +351,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 }
                 const uint32_t dst = smem_u32(smem + OFF_P) + which * TB;  // staging: dK, dV tiles
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    st_shared_v4(dst + sw128_off(row, 4 * h + q), pack_bf16(acc[8 * q], acc[8 * q + 1]),
+                for (int q = 0; q < 2; ++q)
+                    st_shared_v4(dst + sw128_off(row, 2 * g + q), pack_bf16(acc[8 * q], acc[8 * q + 1]),
                                  pack_bf16(acc[8 * q + 2], acc[8 * q + 3]),
                                  pack_bf16(acc[8 * q + 4], acc[8 * q + 5]),
                                  pack_bf16(acc[8 * q + 6], acc[8 * q + 7]));
             }
             fence_proxy_async_smem();
         }
-        named_bar_sync(1, 256);
-        if (!F32 && h == 0 && wg_tid == 0 && ok && *abort == 0) {
+        named_bar_sync(1, 128 * NWG);
+        if (!F32 && g == 0 && wg_tid == 0 && ok && *abort == 0) {
             store_tile(p.dk, part.kframe, p.g, part.o, kt, bh, smem + OFF_P);
             store_tile(p.dv, part.kframe, p.g, part.o, kt, bh, smem + OFF_P + TB);
             bulk_commit();

@@ -59,18 +59,18 @@ __device__ __forceinline__ void store_tile(const FrameMaps &m, int32_t fr, const
     }
 }
 
-// TMA reduce-add of one warp's 32 rows (tile rows 32 q4 .. 32 q4 + 31) x 32 fp32 columns
-// (32 h .. 32 h + 31) of query tile t.  The reduce maps' boxes are 32 rows: {32, 32, 1} in the
-// natural frame, {32, min(Rt, 32), max(1, 32 / Rt), 1} in the grid-column frame.
+// TMA reduce-add of one warp's 32 rows (tile rows 32 q4 .. 32 q4 + 31) x 16 fp32 columns
+// (col0 .. col0 + 15) of query tile t.  The reduce maps' boxes are 16 columns by 32 rows:
+// {16, 32, 1} in the natural frame, {16, min(Rt, 32), max(1, 32 / Rt), 1} in the grid frame.
 __device__ __forceinline__ void reduce_warp_f32(const FrameMaps &m, int32_t fr, const Geom &g, int32_t t,
-                                                int32_t bh, int32_t h, int32_t q4, const void *src)
+                                                int32_t bh, int32_t col0, int32_t q4, const void *src)
 {
     if (fr == FR_NAT) {
-        tma_reduce_add_3d(&m.nat, src, 32 * h, t * TILE + 32 * q4, bh);
+        tma_reduce_add_3d(&m.nat, src, col0, t * TILE + 32 * q4, bh);
     } else {
         const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
         const int32_t rho0 = 32 * q4, a0 = rho0 / g.Rt, r0 = rho0 - a0 * g.Rt;
-        tma_reduce_add_4d(&m.col, src, 32 * h, rt * TILE + r0, grp * g.cpt + a0, bh);
+        tma_reduce_add_4d(&m.col, src, col0, rt * TILE + r0, grp * g.cpt + a0, bh);
     }
 }
 
