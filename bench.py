@@ -45,7 +45,9 @@ FLUSH_BYTES = 256 << 20
 
 # DRAM traffic of the dominant kernel (st_attn_bwd_main) per launch, from an ncu capture, valid
 # only while the kernel sources hash to `src`.  Filled in from profiles/ after a capture.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("fixed_n12288_l128_c32", "08f779797bf1743c"): 173298432,  # profiles/bwd_kernel_fixed_n12288_l128_c32.md
+}
 
 
 def kernel_src_hash() -> str:
