@@ -217,21 +217,33 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             if (ok) tc_fence_after();
             return ok;
         };
-        auto p_phase = [&](int j) {    // P_j = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
+        // Row data of query tile j (interval, -lse, -D).  The loads are issued just before the
+        // wait for S_j: issued any earlier they would sit in front of the proxy fences of the dS
+        // phase, which wait for them.
+        float nlse_n = 0.f, nD_n = 0.f;
+        int32_t lo_n = 1, hi_n = 0;
+        auto prefetch = [&](int j) {
             int32_t lo_abs, hi_abs;
             const int32_t i = row_interval(p.g, part, w.begin + j, row, lo_abs, hi_abs);
-            nlse = 0.f;
-            nD = 0.f;
+            nlse_n = 0.f;
+            nD_n = 0.f;
             if (i >= 0) {
                 const float lse = p.lse[head_base + i];
                 // a row with no allowed key (lse = -inf) has every entry masked to -inf below;
                 // keep its base finite so that -inf + base stays -inf instead of NaN
-                nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
-                nD = -p.delta[head_base + i] * dsc;
+                nlse_n = lse == -INFINITY ? 0.f : -lse * LOG2E;
+                nD_n = -p.delta[head_base + i] * dsc;
             }
             const int32_t base = kt * TILE + CW * g;
-            lo = lo_abs - base;
-            hi = hi_abs - base;
+            lo_n = lo_abs - base;
+            hi_n = hi_abs - base;
+        };
+        auto p_phase = [&](int j) {    // P_j = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
+            prefetch(j);
+            nlse = nlse_n;
+            nD = nD_n;
+            lo = lo_n;
+            hi = hi_n;
             if (!wait_all(&bars->s_full, j & 1)) return;
             tmem_ld32(tS, sv);
             tmem_wait_ld();

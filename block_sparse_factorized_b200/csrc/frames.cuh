@@ -42,15 +42,40 @@ constexpr int32_t TILE = 128;
 enum Frame : int32_t { FR_NAT = 0, FR_COL = 1, FR_SUM = 2 };
 enum Rule : int32_t { RU_BAND = 0, RU_BLOCK = 1, RU_COL = 2, RU_SUM = 3, RU_SUMPREV = 4 };
 
+// Division by a runtime constant d >= 1 as a multiply-high and a shift (valid for 0 <= x < 2^31):
+// with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,  x / d = (umulhi(x, m) + x) >> s.
+struct FastDiv {
+    uint32_t mul, shift;
+};
+
+inline FastDiv make_fastdiv(uint32_t d)
+{
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    const uint64_t m = ((((1ull << s) - d) << 32) / d) + 1;
+    return FastDiv{static_cast<uint32_t>(m), s};
+}
+
+ST_HD int32_t fdiv(int32_t x, FastDiv f)
+{
+#if defined(__CUDA_ARCH__)
+    const uint32_t hi = __umulhi(static_cast<uint32_t>(x), f.mul);
+#else
+    const uint32_t hi = static_cast<uint32_t>((static_cast<uint64_t>(static_cast<uint32_t>(x)) * f.mul) >> 32);
+#endif
+    return static_cast<int32_t>((hi + static_cast<uint32_t>(x)) >> f.shift);
+}
+
 struct Geom {
     int32_t n, l, c;
     int32_t R;        // n / l grid rows
-    int32_t Rt;       // rows per column slot in a column-frame tile
+    int32_t Rt;       // rows per column slot in a column-frame tile (a power of two)
     int32_t cpt;      // column slots per column-frame tile
     int32_t tpc;      // column-frame tiles per column group
     int32_t ngroups;  // column groups
     int32_t upt;      // summary blocks per summary-frame tile (128 / c)
     int32_t pad[3];
+    FastDiv div_l, div_c, div_tpc, div_Rt;  // for the per-row frame arithmetic
 };
 
 struct Part {
@@ -83,13 +108,13 @@ ST_HD int32_t frame_pos(const Geom &g, int32_t fr, int32_t o, int32_t t, int32_t
 {
     if (fr == FR_NAT) return t * TILE + rho;
     if (fr == FR_COL) {
-        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
-        const int32_t a = rho / g.Rt, rr = rho - a * g.Rt;
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
+        const int32_t a = fdiv(rho, g.div_Rt), rr = rho - a * g.Rt;
         const int32_t col = grp * g.cpt + a, r = rt * TILE + rr;
         return (col < g.l && r < g.R) ? r * g.l + col : -1;
     }
     const int32_t kappa = t * TILE + rho;
-    const int32_t u = kappa / g.c, s = kappa - u * g.c;
+    const int32_t u = fdiv(kappa, g.div_c), s = kappa - u * g.c;
     return u < g.R ? u * g.l + (g.l - g.c - o) + s : -1;
 }
 
@@ -106,22 +131,22 @@ ST_HD int32_t row_interval(const Geom &g, const Part &p, int32_t t, int32_t rho,
         hi = i - p.hi_off;
         break;
     case RU_BLOCK:
-        lo = (i / g.l) * g.l;
+        lo = fdiv(i, g.div_l) * g.l;
         hi = i;
         break;
     case RU_COL: {
-        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
-        const int32_t a = rho / g.Rt, rr = rho - a * g.Rt;
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
+        const int32_t a = fdiv(rho, g.div_Rt), rr = rho - a * g.Rt;
         lo = grp * g.tpc * TILE + a * g.Rt;
         hi = lo + rt * TILE + rr;
         break;
     }
     case RU_SUMPREV:
         lo = 0;
-        hi = (i / g.l) * g.c - 1;
+        hi = fdiv(i, g.div_l) * g.c - 1;
         break;
     default: {  // RU_SUM
-        const int32_t blk = i / g.l;
+        const int32_t blk = fdiv(i, g.div_l);
         int32_t w = i - blk * g.l - (g.l - g.c - p.o) + 1;
         w = imax(0, imin(w, g.c));
         lo = 0;

@@ -146,6 +146,10 @@ st_status_t build_exec(st_layout &L)
         g.tpc = 1;
     }
     g.ngroups = (l + g.cpt - 1) / g.cpt;
+    g.div_l = st::make_fastdiv(static_cast<uint32_t>(l));
+    g.div_c = st::make_fastdiv(static_cast<uint32_t>(c > 0 ? c : 1));
+    g.div_tpc = st::make_fastdiv(static_cast<uint32_t>(g.tpc));
+    g.div_Rt = st::make_fastdiv(static_cast<uint32_t>(g.Rt));
     if (L.pat.family == ST_FIXED) {
         if (!is_pow2(c) || c > st::TILE || c > l) return ST_ERR_UNSUPPORTED;
         g.upt = st::TILE / c;

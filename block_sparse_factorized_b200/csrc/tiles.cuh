@@ -37,7 +37,7 @@ __device__ __forceinline__ void load_tile(const FrameMaps &m, int32_t fr, const 
     if (fr == FR_NAT) {
         tma_load_3d(dst, &m.nat, bar, 0, t * TILE, bh);
     } else if (fr == FR_COL) {
-        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
         tma_load_4d(dst, &m.col, bar, 0, rt * TILE, grp * g.cpt, bh);
     } else {
         tma_load_4d(dst, &m.sum, bar, 0, g.l - g.c - o, t * g.upt, bh);
@@ -52,7 +52,7 @@ __device__ __forceinline__ void store_tile(const FrameMaps &m, int32_t fr, const
     if (fr == FR_NAT) {
         tma_store_3d(&m.nat, src, 0, t * TILE, bh);
     } else if (fr == FR_COL) {
-        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
         tma_store_4d(&m.col, src, 0, rt * TILE, grp * g.cpt, bh);
     } else {
         tma_store_4d(&m.sum, src, 0, g.l - g.c - o, t * g.upt, bh);
@@ -68,8 +68,8 @@ __device__ __forceinline__ void reduce_warp_f32(const FrameMaps &m, int32_t fr, 
     if (fr == FR_NAT) {
         tma_reduce_add_3d(&m.nat, src, col0, t * TILE + 32 * q4, bh);
     } else {
-        const int32_t grp = t / g.tpc, rt = t - grp * g.tpc;
-        const int32_t rho0 = 32 * q4, a0 = rho0 / g.Rt, r0 = rho0 - a0 * g.Rt;
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
+        const int32_t rho0 = 32 * q4, a0 = fdiv(rho0, g.div_Rt), r0 = rho0 - a0 * g.Rt;
         tma_reduce_add_4d(&m.col, src, col0, rt * TILE + r0, grp * g.cpt + a0, bh);
     }
 }
