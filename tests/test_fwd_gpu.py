@@ -34,6 +34,8 @@ SMALL = [
     Workload("f_n1024_l256_c8", FIXED, ALTERNATING, 1024, 256, 8, 1, 4),
     Workload("f_single_a2_n512_l32_c4", FIXED, SINGLE_A2, 512, 32, 4, 1, 8),
     Workload("f_merged_n1024_l128_c32", FIXED, MERGED, 1024, 128, 32, 1, 4),
+    # long backward items: summary key tile 0 is read by all 64 query tiles
+    Workload("f_n8192_l128_c32_long", FIXED, ALTERNATING, 8192, 128, 32, 1, 2),
 ]
 
 
@@ -60,7 +62,8 @@ BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
 FP32 = [WORKLOADS["strided_n256_l16_fp32"],
         Workload("f32_fixed_n512_l128_c32", FIXED, ALTERNATING, 512, 128, 32, 1, 4, dtype="fp32"),
         Workload("f32_s_merged_n768_l24", STRIDED, MERGED, 768, 24, 0, 1, 2, dtype="fp32"),
-        Workload("f32_f_merged_n512_l128_c32", FIXED, MERGED, 512, 128, 32, 1, 2, dtype="fp32")]
+        Workload("f32_f_merged_n512_l128_c32", FIXED, MERGED, 512, 128, 32, 1, 2, dtype="fp32"),
+        Workload("f32_fixed_n8192_l128_c32_long", FIXED, SINGLE_A2, 8192, 128, 32, 1, 1, dtype="fp32")]
 
 
 @pytest.mark.parametrize("w", FP32, ids=lambda w: w.name)
