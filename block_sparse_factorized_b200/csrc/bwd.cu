@@ -256,8 +256,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     sv[e] = keep ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
                 }
             }
+            {
+                const uint64_t sc2 = f32x2(sc, sc), nl2 = f32x2(nlse, nlse);
 #pragma unroll
-            for (int e = 0; e < CW; ++e) pr[e] = ex2(fmaf(__uint_as_float(sv[e]), sc, nlse));
+                for (int e = 0; e < CW; e += 2) {
+                    float x0, x1;
+                    f32x2_split(fma2(f32x2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2), x0, x1);
+                    pr[e] = ex2(x0);
+                    pr[e + 1] = ex2(x1);
+                }
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 st_shared_v4(sPg + sw128_off(row, chunk0 + q), pack_bf16(pr[8 * q], pr[8 * q + 1]),
@@ -271,14 +279,18 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             if (!wait_all(&bars->dp_full, j & 1)) return;
             tmem_ld32(tDP, dv);
             tmem_wait_ld();
+            const uint64_t dsc2 = f32x2(dsc, dsc), nD2 = f32x2(nD, nD);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = 8 * q + 2 * e;
-                    pk[e] = pack_bf16(pr[c] * fmaf(__uint_as_float(dv[c]), dsc, nD),
-                                      pr[c + 1] * fmaf(__uint_as_float(dv[c + 1]), dsc, nD));
+                    // dS = P (dP - D) / sqrt(d), two entries per f32x2 instruction
+                    const uint64_t t = fma2(f32x2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), dsc2, nD2);
+                    float d0, d1;
+                    f32x2_split(mul2(f32x2(pr[c], pr[c + 1]), t), d0, d1);
+                    pk[e] = pack_bf16(d0, d1);
                 }
                 st_shared_v4(sDSg + sw128_off(row, chunk0 + q), pk[0], pk[1], pk[2], pk[3]);
             }

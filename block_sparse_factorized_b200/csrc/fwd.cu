@@ -61,20 +61,17 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 128, "barrier block");
 
-// Row max of 64 scores with eight independent partial maxima (short dependency chains, few
-// extra registers).
+// Row max of 64 scores: eight independent partial maxima folded with three-input max (short
+// dependency chains, about one instruction per two scores).
 __device__ __forceinline__ float max64(const uint32_t (&v)[64])
 {
     float a[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(v[e]);
+    for (int e = 0; e < 8; ++e) a[e] = fmaxf(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
 #pragma unroll
-    for (int c = 8; c < 64; ++c) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(v[c]));
-#pragma unroll
-    for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int e = 0; e < w; ++e) a[e] = fmaxf(a[e], a[e + w]);
-    return a[0];
+    for (int c = 16; c < 64; c += 2)
+        a[(c >> 1) & 7] = max3f(a[(c >> 1) & 7], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+    return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
 
 template <bool SPLIT>
@@ -256,14 +253,13 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
             const float m_use = grow ? m_new : m;
             const float alpha = grow ? ex2(m - m_use) : 1.f;  // 0 when nothing was seen yet
             const float nb = (m_use == -INFINITY) ? 0.f : -m_use;
-            float ps[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
+                // p = exp2(s log2e / sqrt(d) - m)
                 const float p0 = ex2(fmaf(__uint_as_float(v[c]), sc, nb));
                 const float p1 = ex2(fmaf(__uint_as_float(v[c + 1]), sc, nb));
-                ps[(c >> 1) & 7] += p0 + p1;
+                ps[(c >> 1) & 3] += p0 + p1;
                 v[c >> 1] = pack_bf16(p0, p1);
             }
             // PV of the previous tile must be done with P_h and O_h before they change
@@ -289,11 +285,7 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 }
                 tmem_wait_st();
             }
-#pragma unroll
-            for (int w2 = 4; w2 >= 1; w2 >>= 1)
-#pragma unroll
-                for (int e = 0; e < w2; ++e) ps[e] += ps[e + w2];
-            l = l * alpha + ps[0];
+            l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
             m = m_use;
             fence_proxy_async_smem();
             tc_fence_before();
