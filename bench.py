@@ -281,9 +281,12 @@ def run_ours(args, rank, world, local):
     def ptr(t):
         return P(t.data_ptr())
 
+    fws_bytes = int(lib.st_attn_fwd_workspace_bytes(ctypes.byref(desc), lay.handle))
+    fws = torch.empty(fws_bytes, dtype=torch.uint8, device=device)
+
     def fwd():
-        _abi.check(lib.st_attn_fwd(ptr(q), ptr(k), ptr(v), lay.handle, ptr(o), ptr(lse), None, 0,
-                                   ctypes.byref(desc), sp), "st_attn_fwd")
+        _abi.check(lib.st_attn_fwd(ptr(q), ptr(k), ptr(v), lay.handle, ptr(o), ptr(lse), ptr(fws),
+                                   fws_bytes, ctypes.byref(desc), sp), "st_attn_fwd")
 
     def prep():
         _abi.check(lib.st_attn_bwd_prepare(ptr(o), ptr(do), lay.handle, ptr(dk), ptr(dv), ptr(ws),

@@ -8,6 +8,10 @@
 
 namespace {
 
+// Forward workspace head: one int32 unit counter per pass (zeroed by every call), padded so the
+// fp32 copies that follow stay 256-byte aligned.
+constexpr size_t FWD_SCHED_BYTES = 256;
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -149,9 +153,9 @@ extern "C" {
 
 size_t st_attn_fwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    if (!desc || !layout || desc->dtype != ST_FP32) return 0;
-    // fp32 I/O: bf16 copies Q_hi, Q_lo, K_hi, K_lo, V_hi
-    return 5 * bf16_copy_bytes(desc);
+    if (!desc || !layout) return 0;
+    // the unit counters of the two passes; fp32 I/O adds bf16 copies Q_hi, Q_lo, K_hi, K_lo, V_hi
+    return FWD_SCHED_BYTES + (desc->dtype == ST_FP32 ? 5 * bf16_copy_bytes(desc) : 0);
 }
 
 size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
@@ -180,11 +184,13 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
     const bool f32 = desc->dtype == ST_FP32;
     st::FwdParams p;
     memset(&p, 0, sizeof(p));
+    if (!workspace || workspace_bytes < st_attn_fwd_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
+    int32_t *sched = static_cast<int32_t *>(workspace);
+    if (cudaMemsetAsync(sched, 0, 2 * sizeof(int32_t), stream) != cudaSuccess) return ST_ERR_CUDA;
     if (f32) {
-        const size_t need = st_attn_fwd_workspace_bytes(desc, layout), cb = bf16_copy_bytes(desc);
-        if (!workspace || workspace_bytes < need) return ST_ERR_WORKSPACE;
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
-        char *w = static_cast<char *>(workspace);
+        const size_t cb = bf16_copy_bytes(desc);
+        char *w = static_cast<char *>(workspace) + FWD_SCHED_BYTES;
         void *qh = w, *ql = w + cb, *kh = w + 2 * cb, *kl = w + 3 * cb, *vh = w + 4 * cb;
         if (!split_copy(q, qh, ql, desc, stream) || !split_copy(k, kh, kl, desc, stream) ||
             !split_copy(v, vh, nullptr, desc, stream))
@@ -196,7 +202,7 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
         p.o_f32 = static_cast<float *>(o);
         p.o_prev_f32 = static_cast<const float *>(o);
     } else if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) ||
-               !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.o, o, L.geom, BH, f.qcol, false)) {
+               !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum)) {
         return ST_ERR_CUDA;
     }
     p.parts = L.d_parts;
@@ -205,11 +211,13 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
     p.g = L.geom;
     p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
     p.lse = lse;
+    if (!f32) p.o = static_cast<uint16_t *>(o);
     p.o_prev = static_cast<const uint16_t *>(o);
     p.err = L.d_err;
     for (int pass = 0; pass < 2; ++pass) {
         p.items = L.d_fwd[pass];
         p.nitems = static_cast<int32_t>(L.fwd_items[pass].size());
+        p.sched = sched + pass;
         if (st::launch_fwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
     return ST_OK;

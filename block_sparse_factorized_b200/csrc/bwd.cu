@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             if (ok && j + 1 < nq) p_phase(j + 1);
             if (ok) drain(j);
         }
-        if (lane == 0) bulk_wait_all();  // every dQ reduce of this warp has landed
+        if (lane == 0) bulk_wait_read_all();  // this warp's dQ reduces have read their staging
         // ------- dK, dV epilogue: one key row per thread, warpgroup g writes columns OW g.. -------
         if (ok) {
             const int32_t pos = frame_pos(p.g, part.kframe, part.o, kt, row);
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             store_tile(p.dk, part.kframe, p.g, part.o, kt, bh, smem + OFF_P);
             store_tile(p.dv, part.kframe, p.g, part.o, kt, bh, smem + OFF_P + TB);
             bulk_commit();
-            bulk_wait_all();
+            bulk_wait_read_all();  // the CTA may leave once the copy engine has read SMEM
         }
     }
     tc_fence_before();

@@ -17,7 +17,7 @@ struct FrameMaps {
 };
 
 struct FwdParams {
-    FrameMaps q, k, v, o;        // o.sum unused
+    FrameMaps q, k, v;
     FrameMaps ql, kl;            // split precision (fp32 I/O): low bf16 parts of Q and K
     const Part *parts;
     const WorkItem *items;
@@ -25,10 +25,12 @@ struct FwdParams {
     Geom g;
     float scale_log2;            // log2(e) / sqrt(d)
     float *lse;                  // [B*H, n]
+    uint16_t *o;                 // [B*H, n, 64] bf16 output, written row by row
     const uint16_t *o_prev;      // merge pass: the output (bf16) written by the first pass
-    float *o_f32;                // fp32 I/O: output written row by row instead of through TMA
+    float *o_f32;                // fp32 I/O: output written row by row
     const float *o_prev_f32;     // fp32 I/O merge pass: the first pass's output
     int32_t *err;                // device error word
+    int32_t *sched;              // unit counter, zero at launch
 };
 
 struct BwdParams {

@@ -167,7 +167,10 @@ ST_API size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout
 
 /* Forward pass.  q, k, v: inputs; o: output; lse: [batch, heads, n] fp32 output.
  * Launches the fused tcgen05 attention kernel (one pass, or two for merged strided heads whose
- * second pass merges by log-sum-exp into the first pass's O and lse). */
+ * second pass merges by log-sum-exp into the first pass's O and lse).
+ * The workspace (st_attn_fwd_workspace_bytes, never 0) starts with the work-unit counters of the
+ * persistent kernel, zeroed on `stream` by every call: calls that run at the same time need
+ * separate workspaces.  fp32 I/O adds the bf16 copies of q, k and v after them. */
 ST_API st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_layout_t *layout,
                         void *o, float *lse, void *workspace, size_t workspace_bytes,
                         const st_desc_t *desc, st_stream_t stream);

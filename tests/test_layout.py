@@ -87,6 +87,11 @@ def test_argument_errors():
     assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
                            ctypes.byref(d), None) == 4
     assert lib.st_layout_check(lay.handle, None) == 4
+    # the forward always takes a workspace: the persistent kernel's unit counters come first
+    d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
+    assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 256
+    d = _abi.st_desc_t(1, 2, 256, 64, 2, 0)
+    assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 256 + 5 * 2 * 256 * 64 * 2
 
 
 def expand_block_row(row_ptr, col_idx, mask_id, masks, qb, B, n):
