@@ -12,6 +12,20 @@ namespace {
 // fp32 copies that follow stay 256-byte aligned.
 constexpr size_t FWD_SCHED_BYTES = 256;
 
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Backward workspace: fp32 dK/dV partial sums of the chunks of split key tiles (one 2 x 128 x 64
+// slot per chunk and batch element) and the item counters of the two passes of the persistent
+// kernel.
+size_t bwd_partial_bytes(const st_desc_t *desc, const st_layout_t *layout)
+{
+    return static_cast<size_t>(layout->bwd_slots) * desc->batch * 2 * 128 * 64 * sizeof(float);
+}
+size_t bwd_counter_bytes(const st_desc_t *, const st_layout_t *)
+{
+    return 2 * sizeof(int32_t);
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -164,7 +178,8 @@ size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *lay
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
     const size_t dq = rows * 64 * sizeof(float);
     const size_t dl = rows * sizeof(float);
-    const size_t base = ((dq + 255) & ~size_t(255)) + ((dl + 255) & ~size_t(255));
+    const size_t base = round256(dq) + round256(dl) + round256(bwd_partial_bytes(desc, layout)) +
+                        round256(bwd_counter_bytes(desc, layout));
     // fp32 I/O adds bf16 copies of Q, K, V and dO for the tensor-core operands
     return desc->dtype == ST_FP32 ? base + 4 * bf16_copy_bytes(desc) : base;
 }
@@ -227,7 +242,9 @@ namespace {
 
 struct BwdWs {
     float *dq_acc, *delta;
-    char *copies;  // fp32 I/O: bf16 Q, K, V, dO
+    float *partials;   // split key tiles: dK/dV partial sums
+    int32_t *counters; // split key tiles: chunks finished
+    char *copies;      // fp32 I/O: bf16 Q, K, V, dO
 };
 
 st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void *workspace,
@@ -236,10 +253,16 @@ st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void
     if (!workspace || workspace_bytes < st_attn_bwd_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
-    ws.dq_acc = static_cast<float *>(workspace);
-    ws.delta = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                         ((rows * 64 * sizeof(float) + 255) & ~size_t(255)));
-    ws.copies = reinterpret_cast<char *>(ws.delta) + ((rows * sizeof(float) + 255) & ~size_t(255));
+    char *w = static_cast<char *>(workspace);
+    ws.dq_acc = reinterpret_cast<float *>(w);
+    w += round256(rows * 64 * sizeof(float));
+    ws.delta = reinterpret_cast<float *>(w);
+    w += round256(rows * sizeof(float));
+    ws.partials = reinterpret_cast<float *>(w);
+    w += round256(bwd_partial_bytes(desc, layout));
+    ws.counters = reinterpret_cast<int32_t *>(w);
+    w += round256(bwd_counter_bytes(desc, layout));
+    ws.copies = w;
     return ST_OK;
 }
 
@@ -271,6 +294,8 @@ st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t
     pre.dk = static_cast<uint16_t *>(dk);
     pre.dv = static_cast<uint16_t *>(dv);
     pre.zero_fill = layout->d_zero_fill;
+    pre.counters = ws.counters;
+    pre.ncounters = 2;
     pre.rows = desc->batch * desc->heads * desc->n;
     pre.n = static_cast<int32_t>(desc->n);
     pre.heads = static_cast<int32_t>(desc->heads);
@@ -309,14 +334,12 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
         dob = c + 3 * cb;
         p.dk_f32 = static_cast<float *>(dk);
         p.dv_f32 = static_cast<float *>(dv);
-        p.dk_prev_f32 = static_cast<const float *>(dk);
-        p.dv_prev_f32 = static_cast<const float *>(dv);
     }
     if (!make_maps_f32(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol)) return ST_ERR_CUDA;
+    if (!f32 && (!make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum)))
+        return ST_ERR_CUDA;
     if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false) ||
         !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum))
-        return ST_ERR_CUDA;
-    if (!f32 && (!make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum)))
         return ST_ERR_CUDA;
     p.parts = L.d_parts;
     p.batch = static_cast<int32_t>(desc->batch);
@@ -327,13 +350,34 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
     p.lse = lse;
     p.delta = ws.delta;
     p.dq_acc = ws.dq_acc;
-    p.dk_prev = static_cast<const uint16_t *>(dk);
-    p.dv_prev = static_cast<const uint16_t *>(dv);
+    p.partials = ws.partials;
+    if (!f32) {
+        p.dk_out = static_cast<uint16_t *>(dk);
+        p.dv_out = static_cast<uint16_t *>(dv);
+    }
     p.err = L.d_err;
     for (int pass = 0; pass < 2; ++pass) {
         p.items = L.d_bwd[pass];
         p.nitems = static_cast<int32_t>(L.bwd_items[pass].size());
+        p.sched = ws.counters + pass;
         if (st::launch_bwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
+        // split key tiles of this pass: the next pass (a merge) reads their dK/dV
+        st::SplitFinishParams sf;
+        memset(&sf, 0, sizeof(sf));
+        sf.partials = ws.partials;
+        sf.recs = L.d_split[pass];
+        sf.parts = L.d_parts;
+        sf.nrecs = static_cast<int32_t>(L.bwd_split_recs[pass].size());
+        sf.batch = p.batch;
+        sf.heads = p.heads;
+        sf.g = L.geom;
+        sf.dk = static_cast<uint16_t *>(dk);
+        sf.dv = static_cast<uint16_t *>(dv);
+        if (f32) {
+            sf.dk_f32 = static_cast<float *>(dk);
+            sf.dv_f32 = static_cast<float *>(dv);
+        }
+        if (st::launch_split_finish(sf, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
     return ST_OK;
 }

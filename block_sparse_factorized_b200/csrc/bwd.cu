@@ -5,19 +5,25 @@
 // then (plain calculus of O = softmax(Q K^T / sqrt d) V over the allowed keys)
 //   dV_j += P_ij dO_i,  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i),  D_i = dO_i . O_i,
 //   dK_j += dS_ij q_i / sqrt(d),  dQ_i += dS_ij k_j / sqrt(d).
-// One CTA owns one 128-key tile (of one part, one batch-head) and walks the contiguous run of
-// query tiles that read it, so dK and dV accumulate in TMEM and are written once; dQ of each
-// (query tile, key tile) pair is added to an fp32 accumulator with vector atomics.
-// Roles:
-//   warp 0      TMA: K and V of the key tile once, then Q and dO per query tile (2-stage ring)
+// A work item is one 128-key tile (of one part, one batch-head) with the contiguous run of query
+// tiles that read it (at most a fixed number: a longer run is split into chunks, whose fp32
+// partials a pass after this kernel sums in chunk order).  dK and dV accumulate in TMEM and are
+// written once per item; dQ of each (query tile, key tile) pair is added to an fp32 accumulator
+// with TMA reduce-adds.
+//
+// The kernel is persistent (one CTA per SM) and claims items, longest first, from a global
+// counter.  K and V have two buffers, so the next item's loads and first S, dP products overlap
+// the current item's last tiles and its dK/dV epilogue.  Roles (576 threads):
+//   warp 0      TMA: K and V of each item (KVS slots), Q and dO per query tile (2-stage ring)
 //   warp 1      MMA issuer: S = Q K^T and dP = dO V^T (TMEM, 128 x 128 fp32 each), then after
 //               the softmax warps wrote P and dS (bf16, SMEM): dV += P^T dO, dK += dS^T Q
 //               (TMEM 128 x 64 each, resident for the whole item) and dQ = dS K (TMEM 128 x 64)
 //   warps 2..17 four warpgroups, one query row per thread, warpgroup g owning score columns
 //               32g..32g+31 (no row reduction is needed here: P comes from the saved lse):
 //               interval mask, P, dS; dQ columns 16g.. staged per warp and added to the fp32
-//               accumulator with a TMA reduce; at the end one key row per thread: dK, dV
-//               columns 16g.. to bf16 and a TMA store.
+//               accumulator with a TMA reduce; at the end of an item one key row per thread:
+//               dK, dV columns 16g.. staged in SMEM for a TMA store (bf16), written row by row
+//               (fp32), or stored as the fp32 partial of a split key tile.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
 #include "tiles.cuh"
 
@@ -26,31 +32,78 @@ namespace {
 
 constexpr uint32_t TB = TILE_BYTES;
 constexpr int NST = 2;                             // Q/dO ring depth
-constexpr uint32_t OFF_K = 0;
-constexpr uint32_t OFF_V = OFF_K + TB;
-constexpr uint32_t OFF_Q = OFF_V + TB;             // NST tiles
+constexpr int NSCHED = 4;                          // claimed-item ring depth
+constexpr int KVS = 2;                             // K/V slots (items in flight)
+constexpr uint32_t OFF_K = 0;                      // KVS slots
+constexpr uint32_t OFF_V = OFF_K + KVS * TB;       // KVS slots
+constexpr uint32_t OFF_Q = OFF_V + KVS * TB;       // NST tiles
 constexpr uint32_t OFF_DO = OFF_Q + NST * TB;      // NST tiles
-constexpr uint32_t OFF_P = OFF_DO + NST * TB;      // 2 halves; dK/dV staging at the end
+constexpr uint32_t OFF_P = OFF_DO + NST * TB;      // 2 halves
 constexpr uint32_t OFF_DS = OFF_P + 2 * TB;        // 2 halves
 constexpr uint32_t OFF_DQ = OFF_DS + 2 * TB;       // dQ staging: 2 x (128 rows x 32 fp32)
 constexpr uint32_t OFF_BAR = OFF_DQ + 2 * TB;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+constexpr uint32_t OFF_ITEMS = OFF_BAR + 256;      // the claimed items' fields, NSCHED entries
+constexpr uint32_t SMEM_BYTES = OFF_ITEMS + NSCHED * 96;
 constexpr int NWG = 4;                             // softmax warpgroups
-constexpr int THREADS = 64 + 128 * NWG;
-constexpr int CW = 128 / NWG;                       // score columns per warpgroup (32)
-constexpr int OW = 64 / NWG;                        // dQ / dK / dV columns per warpgroup (16)
+constexpr int NSM = 128 * NWG;                     // softmax threads
+constexpr int THREADS = 64 + NSM;
+constexpr int CW = 128 / NWG;                      // score columns per warpgroup (32)
+constexpr int OW = 64 / NWG;                       // dQ / dK / dV columns per warpgroup (16)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 320, COL_DQ = 384;
 
 struct Bars {
-    uint64_t kv_full, s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
+    uint64_t kv_full[KVS], kv_empty[KVS];
     uint64_t qdo_full[NST], qdo_empty[NST];
+    uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
+    uint64_t acc_free;             // the epilogue has read dK and dV of the item from TMEM
+    uint64_t stage_full, stage_free;  // bf16 dK/dV staged in the P area / its TMA store has read it
+    uint64_t sched_full[NSCHED], sched_empty[NSCHED];
+    int32_t sched[NSCHED];         // claimed item (index into items x batch), -1 = none left
     uint32_t tmem_base;
     int32_t abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// F32: fp32 I/O -- dK and dV are written row by row in fp32 (the MMAs run on bf16 copies).
+struct Item {
+    WorkItem w;
+    Part part;
+    int32_t b, bh, nq;
+};
+static_assert(sizeof(Item) <= 96, "item slot");
+
+__device__ __forceinline__ Item load_item(const BwdParams &p, int32_t u)
+{
+    Item r;
+    const int32_t item = u / p.batch;
+    r.b = u - item * p.batch;
+    r.w = p.items[item];
+    r.part = p.parts[r.w.part];
+    r.bh = r.b * p.heads + r.part.head;
+    r.nq = r.w.end - r.w.begin;
+    return r;
+}
+
+// The j-th item this CTA processes, as claimed by the producer (its fields are in the shared
+// item slot j % NSCHED until the caller releases it with done_item): -1 when the list is
+// exhausted, -2 when the wait gave up.  Called by the MMA thread (warp_wide false) or by whole
+// softmax warps.
+__device__ __forceinline__ int32_t next_item(Bars *bars, int32_t j, bool warp_wide, volatile int32_t *abort,
+                                             int32_t *err)
+{
+    const int s = j % NSCHED;
+    bool ok = mbar_wait(&bars->sched_full[s], (j / NSCHED) & 1, abort, err);
+    if (warp_wide) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return -2;
+    return *reinterpret_cast<volatile int32_t *>(&bars->sched[s]);
+}
+__device__ __forceinline__ void done_item(Bars *bars, int32_t j, bool warp_wide)
+{
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || (threadIdx.x & 31) == 0) mbar_arrive(&bars->sched_empty[j % NSCHED]);
+}
+
+// F32: fp32 I/O -- dK and dV are written in fp32 (the MMAs run on bf16 copies).
 template <bool F32>
 __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p)
 {
@@ -58,25 +111,29 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BAR);
     volatile int32_t *abort = &bars->abort;
-
-    const int32_t item = blockIdx.x / p.batch, b = blockIdx.x - item * p.batch;
-    const WorkItem w = p.items[item];
-    const Part part = p.parts[w.part];
-    const int32_t bh = b * p.heads + part.head;
-    const int32_t kt = w.tile;
-    const int32_t nq = w.end - w.begin;
+    const int32_t nunits = p.nitems * p.batch;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->dp_full, 1);
-        mbar_init(&bars->p_ready, 128 * NWG);
-        mbar_init(&bars->ds_ready, 128 * NWG);
-        mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 128 * NWG);
+        for (int s = 0; s < KVS; ++s) {
+            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
+        }
         for (int s = 0; s < NST; ++s) {
             mbar_init(&bars->qdo_full[s], 1);
             mbar_init(&bars->qdo_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_ready, NSM);
+        mbar_init(&bars->ds_ready, NSM);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_empty, NSM);
+        mbar_init(&bars->acc_free, NSM);
+        mbar_init(&bars->stage_full, NSM);
+        mbar_init(&bars->stage_free, 1);
+        for (int s = 0; s < NSCHED; ++s) {
+            mbar_init(&bars->sched_full[s], 1);
+            mbar_init(&bars->sched_empty[s], 1 + NSM / 32);  // the MMA thread and each softmax warp
         }
         bars->abort = (smem_u32(smem) & 1023u) ? 1 : 0;
         if (bars->abort) atomicOr(p.err, 2);
@@ -90,32 +147,59 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = bars->tmem_base;
-    const bool run = (*abort == 0) && nq > 0;
+    const bool run = (*abort == 0);
 
+    // Phase bookkeeping shared by every role: I counts items processed by this CTA (K/V slot
+    // I % 2, the dK/dV hand-off), J counts query tiles over all of them (Q/dO ring, per-tile
+    // barriers).
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0 && run) {
-            tma_prefetch(frame_map(p.q, part.qframe));
-            tma_prefetch(frame_map(p.dout, part.qframe));
-            mbar_arrive_expect_tx(&bars->kv_full, 2 * TB);
-            load_tile(p.k, part.kframe, p.g, part.o, kt, bh, smem + OFF_K, &bars->kv_full);
-            load_tile(p.v, part.kframe, p.g, part.o, kt, bh, smem + OFF_V, &bars->kv_full);
-            int j = 0;
-            for (; j < nq; ++j) {
-                const int s = j % NST;
-                if (j >= NST && !mbar_wait(&bars->qdo_empty[s], ((j / NST) - 1) & 1, abort, p.err))
+            tma_prefetch(&p.q.nat);
+            tma_prefetch(&p.dout.nat);
+            tma_prefetch(&p.k.nat);
+            tma_prefetch(&p.v.nat);
+            int32_t I = 0, J = 0;  // K/V loads and Q/dO loads issued
+            bool fail = false;
+            for (int32_t j = 0; !fail; ++j) {
+                // items are claimed from a global counter in list order (longest first) and
+                // broadcast to the other roles through sched[]
+                const int s = j % NSCHED;
+                if (j >= NSCHED && !mbar_wait(&bars->sched_empty[s], ((j / NSCHED) - 1) & 1, abort, p.err))
                     break;
-                mbar_arrive_expect_tx(&bars->qdo_full[s], 2 * TB);
-                load_tile(p.q, part.qframe, p.g, part.o, w.begin + j, bh, smem + OFF_Q + s * TB,
-                          &bars->qdo_full[s]);
-                load_tile(p.dout, part.qframe, p.g, part.o, w.begin + j, bh,
-                          smem + OFF_DO + s * TB, &bars->qdo_full[s]);
+                int32_t u = atomicAdd(p.sched, 1);
+                if (u >= nunits) u = -1;
+                bars->sched[s] = u;
+                Item *slot = reinterpret_cast<Item *>(smem + OFF_ITEMS) + s;
+                if (u >= 0) *slot = load_item(p, u);
+                mbar_arrive(&bars->sched_full[s]);
+                if (u < 0) break;
+                const Item it = *slot;
+                const int ks = I % KVS;
+                if (I >= KVS && !mbar_wait(&bars->kv_empty[ks], ((I / KVS) - 1) & 1, abort, p.err)) break;
+                mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * TB);
+                load_tile(p.k, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_K + ks * TB, &bars->kv_full[ks]);
+                load_tile(p.v, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_V + ks * TB, &bars->kv_full[ks]);
+                ++I;
+                for (int32_t jj = 0; jj < it.nq; ++jj, ++J) {
+                    const int qs = J % NST;
+                    if (J >= NST && !mbar_wait(&bars->qdo_empty[qs], ((J / NST) - 1) & 1, abort, p.err)) {
+                        fail = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->qdo_full[qs], 2 * TB);
+                    load_tile(p.q, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh, smem + OFF_Q + qs * TB,
+                              &bars->qdo_full[qs]);
+                    load_tile(p.dout, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh,
+                              smem + OFF_DO + qs * TB, &bars->qdo_full[qs]);
+                }
             }
             if (*abort) {  // drain the copies still in flight before the CTA leaves
                 volatile int32_t never = 0;
-                mbar_wait(&bars->kv_full, 0, &never, p.err);
-                for (int jj = (j > NST ? j - NST : 0); jj < j; ++jj)
-                    mbar_wait(&bars->qdo_full[jj % NST], (jj / NST) & 1, &never, p.err);
+                for (int32_t i = (I > KVS ? I - KVS : 0); i < I; ++i)
+                    mbar_wait(&bars->kv_full[i % KVS], (i / KVS) & 1, &never, p.err);
+                for (int32_t i = (J > NST ? J - NST : 0); i < J; ++i)
+                    mbar_wait(&bars->qdo_full[i % NST], (i / NST) & 1, &never, p.err);
             }
         }
     } else if (warp == 1) {
@@ -124,66 +208,90 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             constexpr uint32_t id_nn = idesc_bf16(128, 128, false, false);  // S, dP
             constexpr uint32_t id_tt = idesc_bf16(128, 64, true, true);     // dV, dK
             constexpr uint32_t id_kt = idesc_bf16(128, 64, false, true);    // dQ
-            const uint32_t sK = smem_u32(smem + OFF_K), sV = smem_u32(smem + OFF_V);
             const uint32_t sP = smem_u32(smem + OFF_P), sDS = smem_u32(smem + OFF_DS);
-            // Per query tile j the tensor core runs, in order:
-            //   dV += P_j^T dO_j | S_{j+1} | dK += dS_j^T Q_j, dQ_j = dS_j K | dP_{j+1}
-            // so that it computes dV_j and S_{j+1} while the softmax warps build dS_j, and dK_j,
-            // dQ_j, dP_{j+1} while they drain dQ_j and build P_{j+1}.
-            auto issue_s = [&](uint32_t sQ) {  // S = Q K^T (both K-major over d)
+            auto sQ = [&](int32_t t) { return smem_u32(smem + OFF_Q + (t % NST) * TB); };
+            auto sDO = [&](int32_t t) { return smem_u32(smem + OFF_DO + (t % NST) * TB); };
+            // Per query tile t the tensor core runs, in order:
+            //   dV += P_t^T dO_t | S_{t+1} | dK += dS_t^T Q_t, dQ_t = dS_t K | dP_{t+1}
+            // so that it computes dV_t and S_{t+1} while the softmax warps build dS_t, and dK_t,
+            // dQ_t, dP_{t+1} while they drain dQ_t and build P_{t+1}.  An item's first S and dP
+            // follow the previous item's last dQ.
+            auto issue_s = [&](uint32_t q, uint32_t k) {  // S = Q K^T (both K-major over d)
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ss(tbase + COL_S, desc_sw128(sQ + 32 * k, 16, 1024),
-                                desc_sw128(sK + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tbase + COL_S, desc_sw128(q + 32 * kk, 16, 1024),
+                                desc_sw128(k + 32 * kk, 16, 1024), id_nn, kk > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full);
             };
-            auto issue_dp = [&](uint32_t sDO) {  // dP = dO V^T
+            auto issue_dp = [&](uint32_t o, uint32_t v) {  // dP = dO V^T
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ss(tbase + COL_DP, desc_sw128(sDO + 32 * k, 16, 1024),
-                                desc_sw128(sV + 32 * k, 16, 1024), id_nn, k > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tbase + COL_DP, desc_sw128(o + 32 * kk, 16, 1024),
+                                desc_sw128(v + 32 * kk, 16, 1024), id_nn, kk > 0 ? 1u : 0u);
                 mma_commit(&bars->dp_full);
             };
-            bool go = mbar_wait(&bars->kv_full, 0, abort, p.err) &&
-                      mbar_wait(&bars->qdo_full[0], 0, abort, p.err);
-            if (go) {
+            int32_t I = 0, J = 0;
+            bool fail = false;
+            for (int32_t j = 0; !fail; ++j) {
+                const int32_t u = next_item(bars, j, false, abort, p.err);
+                if (u < 0) break;
+                const int32_t nq = (reinterpret_cast<const Item *>(smem + OFF_ITEMS) + j % NSCHED)->nq;
+                const int ks = I % KVS;
+                const uint32_t sK = smem_u32(smem + OFF_K + ks * TB), sV = smem_u32(smem + OFF_V + ks * TB);
+                if (!mbar_wait(&bars->kv_full[ks], (I / KVS) & 1, abort, p.err) ||
+                    !mbar_wait(&bars->qdo_full[J % NST], (J / NST) & 1, abort, p.err))
+                    break;
                 tc_fence_after();
-                issue_s(smem_u32(smem + OFF_Q));
-                issue_dp(smem_u32(smem + OFF_DO));
-            }
-            for (int j = 0; go && j < nq; ++j) {
-                const int s = j % NST, s1 = (j + 1) % NST;
-                const uint32_t sQ = smem_u32(smem + OFF_Q + s * TB);
-                const uint32_t sDO = smem_u32(smem + OFF_DO + s * TB);
-                const bool next = j + 1 < nq;
-                if (!mbar_wait(&bars->p_ready, j & 1, abort, p.err)) break;
-                tc_fence_after();
-                // dV += P^T dO: A = P^T MN-major (two 64-key atoms 16 KB apart), B = dO
-                // MN-major; 16 queries (2048 bytes) per step
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + k * 2048, TB, 1024),
-                                desc_sw128(sDO + k * 2048, TB, 1024), id_tt, (j > 0 || k > 0) ? 1u : 0u);
-                if (next) {  // S of the next query tile: the softmax warps are done reading S_j
-                    if (!mbar_wait(&bars->qdo_full[s1], ((j + 1) / NST) & 1, abort, p.err)) break;
+                issue_s(sQ(J), sK);
+                issue_dp(sDO(J), sV);
+                for (int32_t jj = 0; jj < nq; ++jj) {
+                    const int32_t t = J + jj;
+                    const bool next = jj + 1 < nq;
+                    if (!mbar_wait(&bars->p_ready, t & 1, abort, p.err)) { fail = true; break; }
+                    // the previous item's epilogue must have read dK and dV before they restart
+                    if (jj == 0 && I > 0 && !mbar_wait(&bars->acc_free, (I - 1) & 1, abort, p.err)) {
+                        fail = true;
+                        break;
+                    }
                     tc_fence_after();
-                    issue_s(smem_u32(smem + OFF_Q + s1 * TB));
+                    // dV += P^T dO: A = P^T MN-major (two 64-key atoms 16 KB apart), B = dO
+                    // MN-major; 16 queries (2048 bytes) per step
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + kk * 2048, TB, 1024),
+                                    desc_sw128(sDO(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
+                    if (next) {  // S of the next query tile: the softmax warps are done reading S_t
+                        if (!mbar_wait(&bars->qdo_full[(t + 1) % NST], ((t + 1) / NST) & 1, abort, p.err)) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_s(sQ(t + 1), sK);
+                    }
+                    if (!mbar_wait(&bars->ds_ready, t & 1, abort, p.err) ||
+                        (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort, p.err))) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    // dK += dS^T Q (as dV), dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + kk * 2048, TB, 1024),
+                                    desc_sw128(sQ(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (kk >> 2) * TB + (kk & 3) * 32, 16, 1024),
+                                    desc_sw128(sK + kk * 2048, TB, 1024), id_kt, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars->dq_full);   // also: dK, dV of the item complete on the last tile
+                    mma_commit(&bars->qdo_empty[t % NST]);
+                    if (next) issue_dp(sDO(t + 1), sV);  // dP_t already consumed
                 }
-                if (!mbar_wait(&bars->ds_ready, j & 1, abort, p.err)) break;
-                if (j > 0 && !mbar_wait(&bars->dq_empty, (j - 1) & 1, abort, p.err)) break;
-                tc_fence_after();
-                // dK += dS^T Q (as dV), dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + k * 2048, TB, 1024),
-                                desc_sw128(sQ + k * 2048, TB, 1024), id_tt, (j > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (k >> 2) * TB + (k & 3) * 32, 16, 1024),
-                                desc_sw128(sK + k * 2048, TB, 1024), id_kt, k > 0 ? 1u : 0u);
-                mma_commit(&bars->dq_full);
-                mma_commit(&bars->qdo_empty[s]);
-                if (next) issue_dp(smem_u32(smem + OFF_DO + s1 * TB));  // dP_j already consumed
+                if (fail) break;
+                mma_commit(&bars->kv_empty[ks]);  // K and V of this item are no longer read
+                done_item(bars, j, false);
+                J += nq;
+                ++I;
             }
         }
     } else {
@@ -191,7 +299,6 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         const int g = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
-        const int wg_tid = threadIdx.x - 64 - 128 * g;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
         const uint32_t tS = tbase + COL_S + lane_off + CW * g, tDP = tbase + COL_DP + lane_off + CW * g;
         const uint32_t tDQ = tbase + COL_DQ + lane_off + OW * g;
@@ -202,49 +309,44 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         const uint32_t warp_slot = (g * 4 + q4) * 2048;     // this warp's dQ staging (32 x 64 B)
         const uint32_t sDQw = smem_u32(smem + OFF_DQ) + warp_slot;
         const float sc = p.scale_log2, dsc = p.ds_scale;
-        const size_t head_base = static_cast<size_t>(bh) * p.g.n;
         bool ok = run;
         uint32_t sv[32], dv[32];
-        float pr[CW];                  // P of this row's CW columns, kept from P_j to dS_j
+        float pr[CW];                  // P of this row's CW columns, kept from P_t to dS_t
         float nlse = 0.f, nD = 0.f;    // -lse (log2 units) and -D_i / sqrt(d) of the row
         int32_t lo = 1, hi = 0;        // allowed columns of this slice, relative to the slice
-        // Order per query tile: P_0; then for each j: dS_j, P_{j+1}, drain dQ_j.  Building P_{j+1}
-        // while the tensor core computes dK_j and dQ_j hides their latency.  Buffer safety comes
-        // from commit order: S_{j+1} is issued after dV_j (so s_full(j+1) means P_j was read) and
-        // dP_{j+1} after dK_j, dQ_j (so dp_full(j+1) means dS_j was read).
+        const Item *cur = nullptr;     // the item being processed (its shared slot: the fields
+                                       // are read where needed, to keep registers free)
+        size_t head_base = 0;          // first row of its batch-head
+        int32_t SF = 0;                // dK/dV tiles staged for a TMA store so far
+        bool stage_pending = false;    // the last item's staging (P area) may still be being read
+        // Order per query tile: P_0; then for each t: dS_t, P_{t+1}, drain dQ_t.  Building P_{t+1}
+        // while the tensor core computes dK_t and dQ_t hides their latency.  Buffer safety comes
+        // from commit order: S_{t+1} is issued after dV_t (so s_full(t+1) means P_t was read) and
+        // dP_{t+1} after dK_t, dQ_t (so dp_full(t+1) means dS_t was read).
         auto wait_all = [&](uint64_t *bar, int parity) {
             ok = ok && __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.err));
             if (ok) tc_fence_after();
             return ok;
         };
-        // Row data of query tile j (interval, -lse, -D).  The loads are issued just before the
-        // wait for S_j: issued any earlier they would sit in front of the proxy fences of the dS
-        // phase, which wait for them.
-        float nlse_n = 0.f, nD_n = 0.f;
-        int32_t lo_n = 1, hi_n = 0;
-        auto prefetch = [&](int j) {
+        // Row data of query tile jj of the item (interval, -lse, -D).  The loads are issued just
+        // before the wait for S: issued any earlier they would sit in front of the proxy fences of
+        // the dS phase, which wait for them.
+        auto p_phase = [&](int32_t t, int32_t jj) {  // P_t = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
             int32_t lo_abs, hi_abs;
-            const int32_t i = row_interval(p.g, part, w.begin + j, row, lo_abs, hi_abs);
-            nlse_n = 0.f;
-            nD_n = 0.f;
+            const int32_t i = row_interval(p.g, cur->part, cur->w.begin + jj, row, lo_abs, hi_abs);
+            nlse = 0.f;
+            nD = 0.f;
             if (i >= 0) {
                 const float lse = p.lse[head_base + i];
                 // a row with no allowed key (lse = -inf) has every entry masked to -inf below;
                 // keep its base finite so that -inf + base stays -inf instead of NaN
-                nlse_n = lse == -INFINITY ? 0.f : -lse * LOG2E;
-                nD_n = -p.delta[head_base + i] * dsc;
+                nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
+                nD = -p.delta[head_base + i] * dsc;
             }
-            const int32_t base = kt * TILE + CW * g;
-            lo_n = lo_abs - base;
-            hi_n = hi_abs - base;
-        };
-        auto p_phase = [&](int j) {    // P_j = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
-            prefetch(j);
-            nlse = nlse_n;
-            nD = nD_n;
-            lo = lo_n;
-            hi = hi_n;
-            if (!wait_all(&bars->s_full, j & 1)) return;
+            const int32_t base = cur->w.tile * TILE + CW * g;
+            lo = lo_abs - base;
+            hi = hi_abs - base;
+            if (!wait_all(&bars->s_full, t & 1)) return;
             tmem_ld32(tS, sv);
             tmem_wait_ld();
             if (!(lo <= 0 && hi >= CW - 1)) {
@@ -266,6 +368,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     pr[e + 1] = ex2(x1);
                 }
             }
+            if (stage_pending) {  // the previous item's dK/dV staging (P area) has been read
+                stage_pending = false;
+                if (!wait_all(&bars->stage_free, (SF - 1) & 1)) return;
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 st_shared_v4(sPg + sw128_off(row, chunk0 + q), pack_bf16(pr[8 * q], pr[8 * q + 1]),
@@ -275,8 +381,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             tc_fence_before();
             mbar_arrive(&bars->p_ready);
         };
-        auto ds_phase = [&](int j) {   // dS_j = P (dP - D) / sqrt(d) -> SMEM
-            if (!wait_all(&bars->dp_full, j & 1)) return;
+        auto ds_phase = [&](int32_t t) {  // dS_t = P (dP - D) / sqrt(d) -> SMEM
+            if (!wait_all(&bars->dp_full, t & 1)) return;
             tmem_ld32(tDP, dv);
             tmem_wait_ld();
             const uint64_t dsc2 = f32x2(dsc, dsc), nD2 = f32x2(nD, nD);
@@ -287,9 +393,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 for (int e = 0; e < 4; ++e) {
                     const int c = 8 * q + 2 * e;
                     // dS = P (dP - D) / sqrt(d), two entries per f32x2 instruction
-                    const uint64_t t = fma2(f32x2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), dsc2, nD2);
+                    const uint64_t x = fma2(f32x2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), dsc2, nD2);
                     float d0, d1;
-                    f32x2_split(mul2(f32x2(pr[c], pr[c + 1]), t), d0, d1);
+                    f32x2_split(mul2(f32x2(pr[c], pr[c + 1]), x), d0, d1);
                     pk[e] = pack_bf16(d0, d1);
                 }
                 st_shared_v4(sDSg + sw128_off(row, chunk0 + q), pk[0], pk[1], pk[2], pk[3]);
@@ -298,8 +404,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             tc_fence_before();
             mbar_arrive(&bars->ds_ready);
         };
-        auto drain = [&](int j) {      // dQ_j columns OW g.. : TMEM -> SMEM -> TMA reduce-add
-            if (!wait_all(&bars->dq_full, j & 1)) return;
+        auto drain = [&](int32_t t, int32_t jj) {  // dQ_t columns OW g.. : TMEM -> SMEM -> TMA reduce-add
+            if (!wait_all(&bars->dq_full, t & 1)) return;
             uint32_t dq[16];
             tmem_ld16(tDQ, dq);
             tmem_wait_ld();
@@ -314,82 +420,142 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                reduce_warp_f32(p.dq_red, part.qframe, p.g, w.begin + j, bh, OW * g, q4,
+                reduce_warp_f32(p.dq_red, cur->part.qframe, p.g, cur->w.begin + jj, cur->bh, OW * g, q4,
                                 smem + OFF_DQ + warp_slot);
                 bulk_commit();
             }
         };
-        if (ok) p_phase(0);
-        for (int j = 0; ok && j < nq; ++j) {
-            ds_phase(j);
-            if (ok && j + 1 < nq) p_phase(j + 1);
-            if (ok) drain(j);
-        }
-        if (lane == 0) bulk_wait_read_all();  // this warp's dQ reduces have read their staging
-        // ------- dK, dV epilogue: one key row per thread, warpgroup g writes columns OW g.. -------
-        if (ok) {
-            const int32_t pos = frame_pos(p.g, part.kframe, part.o, kt, row);
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                uint32_t a16[16];
-                tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
-                tmem_wait_ld();
-                float acc[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(a16[e]);
+        int32_t J = 0;  // query tiles processed
+        for (int32_t j = 0; ok; ++j) {
+            const int32_t u = next_item(bars, j, true, abort, p.err);
+            if (u < 0) break;
+            cur = reinterpret_cast<const Item *>(smem + OFF_ITEMS) + j % NSCHED;
+            head_base = static_cast<size_t>(cur->bh) * p.g.n;
+            const int32_t nq = cur->nq;
+            p_phase(J, 0);
+            for (int32_t jj = 0; ok && jj < nq; ++jj) {
+                const int32_t t = J + jj;
+                ds_phase(t);
+                if (ok && jj + 1 < nq) p_phase(t + 1, jj + 1);
+                if (ok) drain(t, jj);
+            }
+            if (!ok) break;
+            // ------- dK, dV of the item: one key row per thread, warpgroup g owns columns OW g.. -------
+            // (the last drain waited for dq_full of the item's last tile, whose commit covers
+            // every dK and dV product of the item).  dK and dV are handled one at a time: the next
+            // item's first dV product waits for its P_0, which these threads build afterwards
+            // anyway, so releasing TMEM early would gain nothing.
+            const int32_t pos = frame_pos(p.g, cur->part.kframe, cur->part.o, cur->w.tile, row);
+            // output of one row slice: add the first pass's values for a merge part (read by this
+            // same thread), round, store
+            auto emit = [&](int which, float (&a)[OW]) {
+                const size_t off = (head_base + pos) * 64 + OW * g;
                 if (F32) {
-                    if (pos >= 0 && *abort == 0) {
-                        const float *pf = which == 0 ? p.dk_prev_f32 : p.dv_prev_f32;
-                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + (head_base + pos) * 64 + OW * g;
-                        if (part.merge) {
-                            const float4 *src = reinterpret_cast<const float4 *>(pf + (head_base + pos) * 64 + OW * g);
+                    float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + off;
+                    if (cur->part.merge) {
+                        const float4 *src = reinterpret_cast<const float4 *>(of);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float4 u = src[q];
-                                acc[4 * q] += u.x;
-                                acc[4 * q + 1] += u.y;
-                                acc[4 * q + 2] += u.z;
-                                acc[4 * q + 3] += u.w;
+                        for (int q = 0; q < OW / 4; ++q) {
+                            const float4 x = src[q];
+                            a[4 * q] += x.x;
+                            a[4 * q + 1] += x.y;
+                            a[4 * q + 2] += x.z;
+                            a[4 * q + 3] += x.w;
+                        }
+                    }
+                    float4 *d4 = reinterpret_cast<float4 *>(of);
+#pragma unroll
+                    for (int q = 0; q < OW / 4; ++q) d4[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                } else {
+                    uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk_out : p.dv_out) + off);
+                    if (cur->part.merge) {
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const uint4 x = d4[q];
+                            const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                a[8 * q + 2 * e] += bf16_lo(xx[e]);
+                                a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
                             }
                         }
-                        float4 *d4 = reinterpret_cast<float4 *>(of);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d4[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
                     }
-                    continue;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q)
+                        d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
+                                           pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
                 }
-                if (part.merge && pos >= 0) {
-                    const uint16_t *prev = which == 0 ? p.dk_prev : p.dv_prev;
-                    const uint4 *src = reinterpret_cast<const uint4 *>(prev + (head_base + pos) * 64 + OW * g);
+            };
+            // Chunk of a split key tile: store the fp32 partial in this chunk's slot (a pass after
+            // the kernel adds the chunks' slots in chunk order and writes dK and dV), in thread
+            // order: uint4 ((which * 4 + q) * 4 + g) * 128 + row, so that each warp store is 512
+            // contiguous bytes.  bf16 output goes through the P area and one TMA store per tile.
+            constexpr size_t SLOT = 2 * 128 * 64;
+            const bool split = cur->w.slot >= 0;
+            const bool staged = !F32 && !split;
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint4 u = src[q];
-                        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+            for (int which = 0; which < 2; ++which) {
+                uint32_t a16[OW];
+                tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
+                tmem_wait_ld();
+                if (*abort != 0) continue;
+                if (split) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.partials + (static_cast<size_t>(cur->w.slot) * p.batch + cur->b) * SLOT);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            acc[8 * q + 2 * e] += bf16_lo(uu[e]);
-                            acc[8 * q + 2 * e + 1] += bf16_hi(uu[e]);
+                    for (int q = 0; q < OW / 4; ++q)
+                        dst[((which * 4 + q) * 4 + g) * 128 + row] = make_uint4(a16[4 * q], a16[4 * q + 1], a16[4 * q + 2], a16[4 * q + 3]);
+                } else {
+                    float a[OW];
+#pragma unroll
+                    for (int e = 0; e < OW; ++e) a[e] = __uint_as_float(a16[e]);
+                    if (F32) {
+                        if (pos >= 0) emit(which, a);
+                    } else {
+                        if (cur->part.merge && pos >= 0) {  // add the first pass's values
+                            const uint4 *src = reinterpret_cast<const uint4 *>((which == 0 ? p.dk_out : p.dv_out) +
+                                                                               (head_base + pos) * 64 + OW * g);
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const uint4 x = src[q];
+                                const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    a[8 * q + 2 * e] += bf16_lo(xx[e]);
+                                    a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
+                                }
+                            }
                         }
+                        const uint32_t dst = smem_u32(smem + OFF_P) + which * TB;  // staging: dK, dV tiles
+#pragma unroll
+                        for (int q = 0; q < 2; ++q)
+                            st_shared_v4(dst + sw128_off(row, 2 * g + q), pack_bf16(a[8 * q], a[8 * q + 1]),
+                                         pack_bf16(a[8 * q + 2], a[8 * q + 3]), pack_bf16(a[8 * q + 4], a[8 * q + 5]),
+                                         pack_bf16(a[8 * q + 6], a[8 * q + 7]));
                     }
                 }
-                const uint32_t dst = smem_u32(smem + OFF_P) + which * TB;  // staging: dK, dV tiles
-#pragma unroll
-                for (int q = 0; q < 2; ++q)
-                    st_shared_v4(dst + sw128_off(row, 2 * g + q), pack_bf16(acc[8 * q], acc[8 * q + 1]),
-                                 pack_bf16(acc[8 * q + 2], acc[8 * q + 3]),
-                                 pack_bf16(acc[8 * q + 4], acc[8 * q + 5]),
-                                 pack_bf16(acc[8 * q + 6], acc[8 * q + 7]));
             }
-            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->acc_free);  // the next item's first dV, dK may overwrite them
+            if (staged) {
+                // the P area is free: dV of the last tile (its last reader) is done (dq_full)
+                fence_proxy_async_smem();
+                mbar_arrive(&bars->stage_full);
+                if (warp == 2 && lane == 0) {
+                    if (mbar_wait(&bars->stage_full, SF & 1, abort, p.err) && *abort == 0) {
+                        store_tile(p.dk, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, smem + OFF_P);
+                        store_tile(p.dv, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, smem + OFF_P + TB);
+                        bulk_commit();
+                        bulk_wait_read_all();  // the next item's P stores may overwrite the staging
+                    }
+                    mbar_arrive(&bars->stage_free);
+                }
+                ++SF;
+            }
+            stage_pending = staged;
+            done_item(bars, j, true);
+            J += nq;
         }
-        named_bar_sync(1, 128 * NWG);
-        if (!F32 && g == 0 && wg_tid == 0 && ok && *abort == 0) {
-            store_tile(p.dk, part.kframe, p.g, part.o, kt, bh, smem + OFF_P);
-            store_tile(p.dv, part.kframe, p.g, part.o, kt, bh, smem + OFF_P + TB);
-            bulk_commit();
-            bulk_wait_read_all();  // the CTA may leave once the copy engine has read SMEM
-        }
+        if (lane == 0) bulk_wait_read_all();  // this warp's dQ reduces have read their staging
     }
     tc_fence_before();
     __syncthreads();
@@ -397,6 +563,18 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tbase, TMEM_COLS);
     }
+}
+
+int sm_count()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
 }
 
 template <bool F32>
@@ -409,8 +587,10 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (p.nitems == 0) return cudaSuccess;
-    bwd_kernel<F32><<<dim3(static_cast<unsigned>(p.nitems) * p.batch), THREADS, SMEM_BYTES, s>>>(p);
+    const int64_t units = static_cast<int64_t>(p.nitems) * p.batch;
+    if (units == 0) return cudaSuccess;
+    const int64_t cap = sm_count();
+    bwd_kernel<F32><<<static_cast<unsigned>(units < cap ? units : cap), THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -1,8 +1,10 @@
 // bwd_aux.cu -- the memory-bound passes around the backward kernel.
-//   bwd_pre:     D_i = dO_i . O_i (fp32), zero the fp32 dQ accumulator, and zero dK/dV of heads
-//                whose keys are not all written by the main kernel (fixed pattern-2 heads read
-//                only summary positions; every other key gets no gradient).
+//   bwd_pre:     D_i = dO_i . O_i (fp32), zero the fp32 dQ accumulator and the split key tiles'
+//                arrival counters, and zero dK/dV of heads whose keys are not all written by the
+//                main kernel (fixed pattern-2 heads read only summary positions; every other key
+//                gets no gradient).
 //   dq_convert:  dQ fp32 accumulator -> output dtype (round to nearest even).
+//   split_finish: dK/dV of the backward's split key tiles from their chunks' fp32 partials.
 //   split:       fp32 tensor -> bf16 high part (round to nearest even) and optionally the bf16
 //                low part x - hi, the operands of the split-precision products of fp32 I/O.
 // Both are HBM-bound: 8 threads per 64-wide row, 16-byte accesses, grid sized to the SM count.
@@ -15,6 +17,8 @@ namespace {
 template <bool F32>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p)
 {
+    for (int32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < p.ncounters; c += gridDim.x * blockDim.x)
+        p.counters[c] = 0;
     const int64_t sub = threadIdx.x & 7;  // eighth of the 64-wide row
     const int64_t nthr_rows = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 3);
     for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 3) + (threadIdx.x >> 3);
@@ -94,6 +98,74 @@ __global__ void __launch_bounds__(256) split_kernel(const SplitParams p)
     }
 }
 
+// One block per (split key tile, batch element): thread t owns row t % 128, columns 32 (t / 128)
+// .. of dK and of dV; the chunks' partials are added in chunk order (a fixed order: the result
+// does not depend on which chunk finished first).  A slot holds, for each of dK, dV, the 16-byte
+// group q (0..3) of the 16-column slice g (0..3) of row r at uint4 ((which * 4 + q) * 4 + g) * 128
+// + r (the order the backward kernel's threads write it in).
+template <bool F32>
+__global__ void __launch_bounds__(256) split_finish_kernel(const SplitFinishParams p)
+{
+    const int32_t rec_i = blockIdx.x / p.batch, b = blockIdx.x - rec_i * p.batch;
+    const SplitRec rec = p.recs[rec_i];
+    const Part part = p.parts[rec.part];
+    const int32_t row = threadIdx.x & 127, c0 = (threadIdx.x >> 7) * 32;
+    const int32_t pos = frame_pos(p.g, part.kframe, part.o, rec.tile, row);
+    if (pos < 0) return;
+    const size_t slot_floats = 2 * 128 * 64;
+    const size_t out = (static_cast<size_t>(b * p.heads + part.head) * p.g.n + pos) * 64 + c0;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+        float a[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) a[e] = 0.f;
+        for (int32_t c = 0; c < rec.nsplit; ++c) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                p.partials + (static_cast<size_t>(rec.first + c) * p.batch + b) * slot_floats);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {  // columns c0 + 4q ..: slice g = c0 / 16 + q / 4, group q % 4
+                const int gg = (c0 >> 4) + (q >> 2), qq = q & 3;
+                const float4 x = src[((which * 4 + qq) * 4 + gg) * 128 + row];
+                a[4 * q] += x.x;
+                a[4 * q + 1] += x.y;
+                a[4 * q + 2] += x.z;
+                a[4 * q + 3] += x.w;
+            }
+        }
+        if (F32) {
+            float4 *d4 = reinterpret_cast<float4 *>((which == 0 ? p.dk_f32 : p.dv_f32) + out);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 v = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                if (part.merge) {  // add the first pass's values
+                    const float4 x = d4[q];
+                    v.x += x.x;
+                    v.y += x.y;
+                    v.z += x.z;
+                    v.w += x.w;
+                }
+                d4[q] = v;
+            }
+        } else {
+            uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk : p.dv) + out);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (part.merge) {
+                    const uint4 x = d4[q];
+                    const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        a[8 * q + 2 * e] += bf16_lo(xx[e]);
+                        a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
+                    }
+                }
+                d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
+                                   pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+            }
+        }
+    }
+}
+
 int sm_count()
 {
     static int n = 0;
@@ -137,6 +209,17 @@ cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s)
 cudaError_t launch_split(const SplitParams &p, cudaStream_t s)
 {
     split_kernel<<<blocks_for((p.elems / 8 + 255) / 256), 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split_finish(const SplitFinishParams &p, bool f32, cudaStream_t s)
+{
+    if (p.nrecs == 0) return cudaSuccess;
+    const unsigned blocks = static_cast<unsigned>(p.nrecs) * p.batch;
+    if (f32)
+        split_finish_kernel<true><<<blocks, 256, 0, s>>>(p);
+    else
+        split_finish_kernel<false><<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -91,7 +91,20 @@ struct Part {
 
 struct WorkItem {          // fwd: tile = query tile, [begin,end) key tiles; bwd: the converse
     int32_t part, tile, begin, end;
+    // bwd only: a key tile whose query run is long is split into chunks processed by separate
+    // CTAs.  slot: this chunk's fp32 partial-sum slot (-1: not split); nsplit: chunks of the key
+    // tile; first: slot of its chunk 0 (chunks use consecutive slots); split: its SplitRec.
+    int32_t slot, nsplit, first, split;
 };
+static_assert(sizeof(WorkItem) == 32, "work item layout");
+
+// A split key tile: its dK/dV are the sum, in chunk order, of slots first .. first + nsplit - 1.
+struct SplitRec {
+    int32_t part, tile, first, nsplit;
+};
+
+// Longest query run one backward CTA walks; longer runs are split into near-equal chunks.
+constexpr int32_t BWD_CHUNK = 32;
 
 ST_HD int32_t imin(int32_t a, int32_t b) { return a < b ? a : b; }
 ST_HD int32_t imax(int32_t a, int32_t b) { return a > b ? a : b; }

@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                     break;
                 }
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    st_shared_v4(sPh + sw128_off(row, j), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(sPh + sw128_off(row, c), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
                     // rescale this half's partial O (PV of this tile waits for p_full)
                     uint32_t o[32];

@@ -35,7 +35,7 @@ struct FwdParams {
 
 struct BwdParams {
     FrameMaps q, k, v, dout;
-    FrameMaps dk, dv;            // stores (sum used for compacted keys)
+    FrameMaps dk, dv;            // bf16 I/O: dK, dV tile stores (sum used for compacted keys)
     FrameMaps dq_red;            // fp32 dQ accumulator in the query frames, box 32 columns wide
                                  // (reduce-add target; nat and col only)
     const Part *parts;
@@ -47,10 +47,10 @@ struct BwdParams {
     const float *lse;            // [B*H, n] natural-log lse of the forward
     const float *delta;          // [B*H, n] D_i = dO_i . O_i
     float *dq_acc;               // [B*H, n, 64] fp32, zeroed before the main kernel
-    const uint16_t *dk_prev;     // merge pass: dK, dV written by the first pass (bf16)
-    const uint16_t *dv_prev;
+    float *partials;             // [slots, B, 2, 128, 64] fp32 dK/dV partials of split key tiles
+    int32_t *sched;              // item counter of this pass, zeroed before the main kernel
+    uint16_t *dk_out, *dv_out;   // bf16 I/O: dK, dV [B*H, n, 64], written row by row
     float *dk_f32, *dv_f32;      // fp32 I/O: outputs written row by row
-    const float *dk_prev_f32, *dv_prev_f32;
     int32_t *err;
 };
 
@@ -62,6 +62,8 @@ struct PreParams {
     float *dq_acc;               // [B*H, n, 64] zeroed here
     uint16_t *dk, *dv;           // zero-filled for heads flagged in zero_fill
     const int32_t *zero_fill;    // [H]
+    int32_t *counters;           // zeroed here
+    int32_t ncounters;
     int64_t rows;                // B*H*n
     int32_t n, heads;
 };
@@ -71,6 +73,18 @@ struct ConvParams {
     uint16_t *dq;
     float *dq_f32;               // fp32 I/O: plain copy instead of rounding to bf16
     int64_t elems;
+};
+
+// dK/dV of split key tiles: sum of the chunks' fp32 partials in chunk order, plus the first
+// pass's values for a merge part, written at the tile's rows.
+struct SplitFinishParams {
+    const float *partials;       // [slots, B, 2, 128, 64]
+    const SplitRec *recs;
+    const Part *parts;
+    int32_t nrecs, batch, heads;
+    Geom g;
+    uint16_t *dk, *dv;           // bf16 I/O
+    float *dk_f32, *dv_f32;      // fp32 I/O
 };
 
 // fp32 -> bf16 hi (round to nearest even) and, if lo != nullptr, lo = bf16(x - hi)
@@ -85,5 +99,6 @@ cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_split(const SplitParams &p, cudaStream_t s);
+cudaError_t launch_split_finish(const SplitFinishParams &p, bool f32, cudaStream_t s);
 
 }  // namespace st

@@ -198,6 +198,10 @@ st_status_t build_exec(st_layout &L)
     for (auto &p : L.parts) max_q = std::max(max_q, p.nq);
     L.fwd_item_of.assign(L.parts.size() * static_cast<size_t>(max_q), -1);
     for (int a = 0; a < 2; ++a) { L.fwd_items[a].clear(); L.bwd_items[a].clear(); }
+    L.bwd_slots = 0;
+    L.bwd_splits = 0;
+    L.bwd_split_recs[0].clear();
+    L.bwd_split_recs[1].clear();
     L.exec_tiles = 0;
     L.allowed_pairs = 0;
     std::vector<std::vector<st::WorkItem>> fwd_by_part(L.parts.size());
@@ -214,7 +218,7 @@ st_status_t build_exec(st_layout &L)
                 tmin = std::min(tmin, lo / st::TILE);
                 tmax = std::max(tmax, hi / st::TILE);
             }
-            st::WorkItem w{static_cast<int32_t>(pi), qt, tmax < 0 ? 0 : tmin, tmax < 0 ? 0 : tmax + 1};
+            st::WorkItem w{static_cast<int32_t>(pi), qt, tmax < 0 ? 0 : tmin, tmax < 0 ? 0 : tmax + 1, -1, 1, -1, -1};
             L.exec_tiles += w.end - w.begin;
             fwd_by_part[pi].push_back(w);
         }
@@ -234,7 +238,23 @@ st_status_t build_exec(st_layout &L)
                 const auto &w = fwd_by_part[pi][qt];
                 if (!(w.begin <= kt && kt < w.end)) return ST_ERR_INTERNAL;  // not contiguous
             }
-            L.bwd_items[p.merge].push_back(st::WorkItem{static_cast<int32_t>(pi), kt, qmin[kt], qmax[kt] + 1});
+            const int32_t len = qmax[kt] + 1 - qmin[kt];
+            if (len <= st::BWD_CHUNK) {
+                L.bwd_items[p.merge].push_back(
+                    st::WorkItem{static_cast<int32_t>(pi), kt, qmin[kt], qmax[kt] + 1, -1, 1, -1, -1});
+                continue;
+            }
+            // near-equal chunks, each with its own partial-sum slot, sharing one counter
+            const int32_t nch = (len + st::BWD_CHUNK - 1) / st::BWD_CHUNK;
+            for (int32_t ch = 0; ch < nch; ++ch) {
+                const int32_t b0 = qmin[kt] + static_cast<int32_t>(static_cast<int64_t>(len) * ch / nch);
+                const int32_t b1 = qmin[kt] + static_cast<int32_t>(static_cast<int64_t>(len) * (ch + 1) / nch);
+                L.bwd_items[p.merge].push_back(st::WorkItem{static_cast<int32_t>(pi), kt, b0, b1,
+                                                            L.bwd_slots + ch, nch, L.bwd_slots, L.bwd_splits});
+            }
+            L.bwd_split_recs[p.merge].push_back(st::SplitRec{static_cast<int32_t>(pi), kt, L.bwd_slots, nch});
+            L.bwd_slots += nch;
+            L.bwd_splits += 1;
         }
         for (const auto &w : fwd_by_part[pi]) {
             L.fwd_item_of[pi * static_cast<size_t>(max_q) + w.tile] = 0;
@@ -355,10 +375,12 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
     const size_t nb0 = L->bwd_items[0].size() * sizeof(st::WorkItem);
     const size_t nb1 = L->bwd_items[1].size() * sizeof(st::WorkItem);
     const size_t nz = L->head_zero_fill.size() * sizeof(int32_t);
+    const size_t ns0 = L->bwd_split_recs[0].size() * sizeof(st::SplitRec);
+    const size_t ns1 = L->bwd_split_recs[1].size() * sizeof(st::SplitRec);
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     const size_t off_f0 = up(np), off_f1 = off_f0 + up(nf0), off_b0 = off_f1 + up(nf1),
-                 off_b1 = off_b0 + up(nb0), off_z = off_b1 + up(nb1), off_e = off_z + up(nz),
-                 total = off_e + 256;
+                 off_b1 = off_b0 + up(nb0), off_z = off_b1 + up(nb1), off_s0 = off_z + up(nz),
+                 off_s1 = off_s0 + up(ns0), off_e = off_s1 + up(ns1), total = off_e + 256;
     if (!L->uploaded) {
         if (cudaMalloc(&L->d_buf, total) != cudaSuccess) return ST_ERR_OOM;
         if (cudaMemsetAsync(L->d_buf, 0, total, stream) != cudaSuccess) return ST_ERR_CUDA;
@@ -370,6 +392,8 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
         L->d_bwd[0] = reinterpret_cast<st::WorkItem *>(b + off_b0);
         L->d_bwd[1] = reinterpret_cast<st::WorkItem *>(b + off_b1);
         L->d_zero_fill = reinterpret_cast<int32_t *>(b + off_z);
+        L->d_split[0] = reinterpret_cast<st::SplitRec *>(b + off_s0);
+        L->d_split[1] = reinterpret_cast<st::SplitRec *>(b + off_s1);
         L->d_err = reinterpret_cast<int32_t *>(b + off_e);
     }
     auto cp = [&](void *dst, const void *src, size_t bytes) {
@@ -377,7 +401,8 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
     };
     if (!cp(L->d_parts, L->parts.data(), np) || !cp(L->d_fwd[0], L->fwd_items[0].data(), nf0) ||
         !cp(L->d_fwd[1], L->fwd_items[1].data(), nf1) || !cp(L->d_bwd[0], L->bwd_items[0].data(), nb0) ||
-        !cp(L->d_bwd[1], L->bwd_items[1].data(), nb1) || !cp(L->d_zero_fill, L->head_zero_fill.data(), nz))
+        !cp(L->d_bwd[1], L->bwd_items[1].data(), nb1) || !cp(L->d_zero_fill, L->head_zero_fill.data(), nz) ||
+        !cp(L->d_split[0], L->bwd_split_recs[0].data(), ns0) || !cp(L->d_split[1], L->bwd_split_recs[1].data(), ns1))
         return ST_ERR_CUDA;
     L->uploaded = true;
     return ST_OK;

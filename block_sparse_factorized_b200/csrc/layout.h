@@ -29,6 +29,8 @@ struct st_layout {
     std::vector<int32_t> head_zero_fill;   // 1: some key of this head is read by no pass-0 part
     std::vector<st::WorkItem> fwd_items[2], bwd_items[2];
     int32_t passes = 1;
+    int32_t bwd_slots = 0, bwd_splits = 0;  // partial-sum slots and split key tiles (bwd)
+    std::vector<st::SplitRec> bwd_split_recs[2];  // split key tiles of each pass
     int64_t exec_tiles = 0, allowed_pairs = 0;
     std::vector<int32_t> fwd_item_of;      // part * max_tiles + q tile -> fwd item index
 
@@ -40,5 +42,6 @@ struct st_layout {
     st::WorkItem *d_fwd[2] = {nullptr, nullptr};
     st::WorkItem *d_bwd[2] = {nullptr, nullptr};
     int32_t *d_zero_fill = nullptr;
+    st::SplitRec *d_split[2] = {nullptr, nullptr};
     int32_t *d_err = nullptr;
 };
