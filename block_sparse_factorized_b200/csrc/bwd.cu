@@ -57,6 +57,7 @@ struct Bars {
     uint64_t qdo_full[NST], qdo_empty[NST];
     uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
     uint64_t acc_free;             // the epilogue has read dK and dV of the item from TMEM
+    uint64_t mma_idle;             // every MMA this CTA issued has completed (before teardown)
     uint64_t stage_full, stage_free;  // bf16 dK/dV staged in the P area / its TMA store has read it
     uint64_t sched_full[NSCHED], sched_empty[NSCHED];
     int32_t sched[NSCHED];         // claimed item (index into items x batch), -1 = none left
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         mbar_init(&bars->acc_free, NSM);
         mbar_init(&bars->stage_full, NSM);
         mbar_init(&bars->stage_free, 1);
+        mbar_init(&bars->mma_idle, 1);
         for (int s = 0; s < NSCHED; ++s) {
             mbar_init(&bars->sched_full[s], 1);
             mbar_init(&bars->sched_empty[s], 1 + NSM / 32);  // the MMA thread and each softmax warp
@@ -293,6 +295,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 J += nq;
                 ++I;
             }
+            // no product may still be running when TMEM is released (also after an abort)
+            mma_commit(&bars->mma_idle);
+            volatile int32_t never = 0;
+            mbar_wait(&bars->mma_idle, 0, &never, p.err);
         }
     } else {
         // ------- P, dS, dQ drain, epilogue (warps 2..: warpgroup g owns score columns CW g..) -------

@@ -64,6 +64,7 @@ struct Plan {
 struct Bars {
     uint64_t q_full, q_empty, s_full, s_free, o_done, o_free;
     uint64_t st_full, st_read;   // epilogue (m, l) exchange between the two warpgroups
+    uint64_t mma_idle;           // every MMA this CTA issued has completed (before teardown)
     uint64_t p_full[2], pv_done[2];
     uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
     uint64_t sched_full[NSCHED], sched_empty[NSCHED];
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
         mbar_init(&bars->o_free, 256);
         mbar_init(&bars->st_full, 256);
         mbar_init(&bars->st_read, 256);
+        mbar_init(&bars->mma_idle, 1);
         for (int h = 0; h < 2; ++h) {
             mbar_init(&bars->p_full[h], 128);
             mbar_init(&bars->pv_done[h], 1);
@@ -323,6 +325,10 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 T += U.nkt;
                 ++kq;
             }
+            // no product may still be running when TMEM is released (also after an abort)
+            mma_commit(&bars->mma_idle);
+            volatile int32_t never = 0;
+            mbar_wait(&bars->mma_idle, 0, &never, p.err);
         }
     } else {
         // ---------------- softmax of one key half + epilogue (warps 2..9) ----------------
