@@ -44,9 +44,9 @@ TILE = 128
 FLUSH_BYTES = 256 << 20
 
 # DRAM traffic of the dominant kernel (st_attn_bwd_main) per launch, from an ncu capture, valid
-# only while the kernel sources hash to `src`.  Filled in from profiles/ after a capture.
+# only while the kernel sources hash to `src`.  Filled in by hand after a capture.
 NCU_TRAFFIC = {
-    ("fixed_n12288_l128_c32", "08f779797bf1743c"): 173298432,  # profiles/bwd_kernel_fixed_n12288_l128_c32.md
+    ("fixed_n12288_l128_c32", "b7625419d639b6a3"): 193122048,  # dram read + write, --set full capture
 }
 
 
@@ -206,6 +206,23 @@ def step_flops(w, info):
     return fwd * 3.5, fwd * 2.5, info["allowed_pairs"] * w.batch * 4 * w.d * 3.5
 
 
+def step_bytes(w, lay):
+    """Algorithmic HBM bytes of one forward and one backward pass (each tensor touched once):
+    forward Q, O, the K and V rows some query reads, lse; backward adds dO, D, dQ and full dK,
+    dV writes.  A fixed-pattern summary head (kind fA2) reads only n / l * c key rows."""
+    import block_sparse_factorized_b200 as bsf
+    row = w.d * (4 if w.dtype == "fp32" else 2)
+    rows = w.batch * w.heads * w.n
+    used = 0
+    for h in range(w.heads):
+        kind, _ = lay.head_kind(h)
+        used += (w.n // w.l) * w.c if kind == bsf.ST_KIND_FA2 else w.n
+    used *= w.batch
+    fwd = 2 * rows * row + 2 * used * row + rows * 4
+    bwd = fwd + rows * row + rows * 4 + 3 * rows * row
+    return fwd, bwd
+
+
 def layout_info_host(w):
     import block_sparse_factorized_b200 as bsf
     return bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
@@ -328,15 +345,28 @@ def run_ours(args, rank, world, local):
     ms_local = statistics.mean(t_step)
     ms = max_over_ranks(ms_local, world, device)
     value = flops * world / (ms / 1e3) / 1e12
-    launches_per_step = 2 * info["passes"] + 2
+    # fwd per pass; bwd: prepare, the main kernel per pass, a summing pass per split pass, convert
+    launches_per_step = 2 * info["passes"] + 2 + info["split_passes"]
     peaks = measured_peaks()
     main_ms = statistics.mean(t_main)
     achieved = bwd_flops / (main_ms / 1e3) / 1e12
     src = kernel_src_hash()
     tr = NCU_TRAFFIC.get((w.name, src))
-    roofline = {"kernel": "st_attn_bwd_main (bwd_kernel)", "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": tr, "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
+    fwd_bytes, bwd_bytes = step_bytes(w, lay)
+    hbm = {"bytes_fwd": fwd_bytes, "bytes_bwd": bwd_bytes,
+           "achieved_gbs": (fwd_bytes + bwd_bytes) / (ms / 1e3) / 1e9, "peak_gbs": peaks["hbm_gbs"]}
+    hbm["frac"] = hbm["achieved_gbs"] / peaks["hbm_gbs"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)  # flop per byte
+    if flops / (fwd_bytes + bwd_bytes) >= ridge:
+        roofline = {"kernel": "st_attn_bwd_main (bwd_kernel)", "bound": "tensor", "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": tr, "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
+    else:  # below the ridge point: the backward kernel's own bytes against the copy bandwidth
+        bwd_kernel_bytes = bwd_bytes - fwd_bytes // 2  # O is read by the prepare pass, not the kernel
+        gbs = bwd_kernel_bytes / (main_ms / 1e3) / 1e9
+        roofline = {"kernel": "st_attn_bwd_main (bwd_kernel)", "bound": "hbm", "achieved": gbs,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                    "traffic": tr, "peak_source": f"{peaks['source']} copy bandwidth (MEASURED_PEAKS.json)"}
 
     e2e = None
     if not args.no_e2e:
@@ -362,7 +392,7 @@ def run_ours(args, rank, world, local):
         "breakdown_ms": {"fwd": statistics.mean(t_fwd), "bwd_prepare": statistics.mean(t_prep),
                          "bwd_main": main_ms, "bwd_finish": statistics.mean(t_fin)},
         "fwd_tflops": flops / 3.5 / (statistics.mean(t_fwd) / 1e3) / 1e12,
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "hbm": hbm, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         "exec_tiles": info["exec_tiles"] * w.batch, "kernel_src": src,
     }

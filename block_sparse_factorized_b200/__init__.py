@@ -107,7 +107,7 @@ class Layout:
         h = getattr(self, "_h", None)
         if h is not None and h.value:
             self._lib.st_layout_destroy(h)
-            self._h = _c.c_void_p()
+            h.value = None  # (at interpreter exit the ctypes module may already be gone)
 
 
 def _desc(q: torch.Tensor) -> _abi.st_desc_t:

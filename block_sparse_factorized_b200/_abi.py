@@ -51,7 +51,7 @@ class st_desc_t(ctypes.Structure):
 class st_layout_info_t(ctypes.Structure):
     _fields_ = [("fwd_items", ctypes.c_int64), ("exec_tiles", ctypes.c_int64),
                 ("bwd_items", ctypes.c_int64), ("allowed_pairs", ctypes.c_int64),
-                ("passes", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("passes", ctypes.c_int32), ("split_passes", ctypes.c_int32)]
 
 
 _lib = None

@@ -98,70 +98,77 @@ __global__ void __launch_bounds__(256) split_kernel(const SplitParams p)
     }
 }
 
-// One block per (split key tile, batch element): thread t owns row t % 128, columns 32 (t / 128)
-// .. of dK and of dV; the chunks' partials are added in chunk order (a fixed order: the result
-// does not depend on which chunk finished first).  A slot holds, for each of dK, dV, the 16-byte
-// group q (0..3) of the 16-column slice g (0..3) of row r at uint4 ((which * 4 + q) * 4 + g) * 128
-// + r (the order the backward kernel's threads write it in).
+// One block of 512 threads per (split key tile, batch element, matrix): thread t owns row t % 128,
+// columns 16 (t / 128) .. of dK or dV; the chunks' partials are added in chunk order (a fixed
+// order: the result does not depend on which chunk finished first), up to four chunks' loads in
+// flight at a time.  A slot holds, for each of dK, dV, the 16-byte group q (0..3) of the
+// 16-column slice g (0..3) of row r at uint4 ((which * 4 + q) * 4 + g) * 128 + r (the order the
+// backward kernel's threads write it in, so that each warp reads 512 contiguous bytes here).
 template <bool F32>
-__global__ void __launch_bounds__(256) split_finish_kernel(const SplitFinishParams p)
+__global__ void __launch_bounds__(512) split_finish_kernel(const SplitFinishParams p)
 {
-    const int32_t rec_i = blockIdx.x / p.batch, b = blockIdx.x - rec_i * p.batch;
+    const int32_t which = blockIdx.x & 1, rb = blockIdx.x >> 1;
+    const int32_t rec_i = rb / p.batch, b = rb - rec_i * p.batch;
     const SplitRec rec = p.recs[rec_i];
     const Part part = p.parts[rec.part];
-    const int32_t row = threadIdx.x & 127, c0 = (threadIdx.x >> 7) * 32;
+    const int32_t row = threadIdx.x & 127, g = threadIdx.x >> 7;
     const int32_t pos = frame_pos(p.g, part.kframe, part.o, rec.tile, row);
     if (pos < 0) return;
-    const size_t slot_floats = 2 * 128 * 64;
-    const size_t out = (static_cast<size_t>(b * p.heads + part.head) * p.g.n + pos) * 64 + c0;
+    constexpr size_t SLOT4 = 2 * 128 * 64 / 4;  // a slot, in float4
+    float a[16];
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-        float a[32];
+    for (int e = 0; e < 16; ++e) a[e] = 0.f;
+    const float4 *base = reinterpret_cast<const float4 *>(p.partials) + ((which * 4) * 4 + g) * 128 + row;
+    for (int32_t c0 = 0; c0 < rec.nsplit; c0 += 4) {
+        float4 x[4][4];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) a[e] = 0.f;
-        for (int32_t c = 0; c < rec.nsplit; ++c) {
-            const float4 *src = reinterpret_cast<const float4 *>(
-                p.partials + (static_cast<size_t>(rec.first + c) * p.batch + b) * slot_floats);
+        for (int c = 0; c < 4; ++c)
+            if (c0 + c < rec.nsplit) {
+                const float4 *src = base + (static_cast<size_t>(rec.first + c0 + c) * p.batch + b) * SLOT4;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {  // columns c0 + 4q ..: slice g = c0 / 16 + q / 4, group q % 4
-                const int gg = (c0 >> 4) + (q >> 2), qq = q & 3;
-                const float4 x = src[((which * 4 + qq) * 4 + gg) * 128 + row];
-                a[4 * q] += x.x;
-                a[4 * q + 1] += x.y;
-                a[4 * q + 2] += x.z;
-                a[4 * q + 3] += x.w;
+                for (int q = 0; q < 4; ++q) x[c][q] = src[q * 4 * 128];
             }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (c0 + c < rec.nsplit)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    a[4 * q] += x[c][q].x;
+                    a[4 * q + 1] += x[c][q].y;
+                    a[4 * q + 2] += x[c][q].z;
+                    a[4 * q + 3] += x[c][q].w;
+                }
+    }
+    const size_t out = (static_cast<size_t>(b * p.heads + part.head) * p.g.n + pos) * 64 + 16 * g;
+    if (F32) {
+        float4 *d4 = reinterpret_cast<float4 *>((which == 0 ? p.dk_f32 : p.dv_f32) + out);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 v = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+            if (part.merge) {  // add the first pass's values
+                const float4 y = d4[q];
+                v.x += y.x;
+                v.y += y.y;
+                v.z += y.z;
+                v.w += y.w;
+            }
+            d4[q] = v;
         }
-        if (F32) {
-            float4 *d4 = reinterpret_cast<float4 *>((which == 0 ? p.dk_f32 : p.dv_f32) + out);
+    } else {
+        uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk : p.dv) + out);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 v = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-                if (part.merge) {  // add the first pass's values
-                    const float4 x = d4[q];
-                    v.x += x.x;
-                    v.y += x.y;
-                    v.z += x.z;
-                    v.w += x.w;
+        for (int q = 0; q < 2; ++q) {
+            if (part.merge) {
+                const uint4 y = d4[q];
+                const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    a[8 * q + 2 * e] += bf16_lo(yy[e]);
+                    a[8 * q + 2 * e + 1] += bf16_hi(yy[e]);
                 }
-                d4[q] = v;
             }
-        } else {
-            uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk : p.dv) + out);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (part.merge) {
-                    const uint4 x = d4[q];
-                    const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        a[8 * q + 2 * e] += bf16_lo(xx[e]);
-                        a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
-                    }
-                }
-                d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
-                                   pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
-            }
+            d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
+                               pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
         }
     }
 }
@@ -215,11 +222,11 @@ cudaError_t launch_split(const SplitParams &p, cudaStream_t s)
 cudaError_t launch_split_finish(const SplitFinishParams &p, bool f32, cudaStream_t s)
 {
     if (p.nrecs == 0) return cudaSuccess;
-    const unsigned blocks = static_cast<unsigned>(p.nrecs) * p.batch;
+    const unsigned blocks = static_cast<unsigned>(p.nrecs) * p.batch * 2;
     if (f32)
-        split_finish_kernel<true><<<blocks, 256, 0, s>>>(p);
+        split_finish_kernel<true><<<blocks, 512, 0, s>>>(p);
     else
-        split_finish_kernel<false><<<blocks, 256, 0, s>>>(p);
+        split_finish_kernel<false><<<blocks, 512, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -442,6 +442,7 @@ st_status_t st_layout_info(const st_layout_t *L, st_layout_info_t *info)
     info->exec_tiles = L->exec_tiles;
     info->allowed_pairs = L->allowed_pairs;
     info->passes = L->passes;
+    info->split_passes = (L->bwd_split_recs[0].empty() ? 0 : 1) + (L->bwd_split_recs[1].empty() ? 0 : 1);
     return ST_OK;
 }
 

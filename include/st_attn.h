@@ -145,7 +145,8 @@ typedef struct {
     int64_t bwd_items;      /* backward work items (key tiles over all heads and passes) */
     int64_t allowed_pairs;  /* sum over heads and rows of |A(h, i)| */
     int32_t passes;         /* 1, or 2 for merged strided heads (band part, then grid part) */
-    int32_t reserved;
+    int32_t split_passes;   /* passes with a key tile whose query run is split over several CTAs
+                               (each adds one short summing launch to the backward pass) */
 } st_layout_info_t;
 ST_API st_status_t st_layout_info(const st_layout_t *layout, st_layout_info_t *info);
 
