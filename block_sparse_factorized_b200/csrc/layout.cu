@@ -350,7 +350,6 @@ st_status_t st_layout_build(const st_pattern_t *pattern, int64_t n, int32_t l, i
             }
             L->head_plan[h] = found;
         }
-        for (auto &np : L->plans) build_nat_plan(np, n, l, L->c, block);
         const st_status_t es = build_exec(*L);
         if (es == ST_ERR_INTERNAL) { delete L; return ST_ERR_INTERNAL; }
         L->exec_ok = (es == ST_OK);
@@ -421,7 +420,16 @@ st_status_t st_layout_export(const st_layout_t *L, int32_t head, const int32_t *
                              const uint32_t **masks, int32_t *n_qblk, int32_t *nnz, int32_t *n_masks)
 {
     if (!L || head < 0 || head >= L->pat.num_heads) return ST_ERR_INVALID_ARG;
-    const NatPlan &P = L->plans[L->head_plan[head]];
+    NatPlan &P = L->plans[L->head_plan[head]];
+    try {
+        std::lock_guard<std::mutex> lock(L->plans_mu);
+        if (!P.built) {
+            build_nat_plan(P, L->n, L->l, L->c, L->block);
+            P.built = true;
+        }
+    } catch (const std::bad_alloc &) {
+        return ST_ERR_OOM;
+    }
     if (row_ptr) *row_ptr = P.row_ptr.data();
     if (col_idx) *col_idx = P.col_idx.data();
     if (mask_id) *mask_id = P.mask_id.data();

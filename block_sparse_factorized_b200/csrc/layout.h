@@ -2,6 +2,7 @@
 #pragma once
 #include <stdint.h>
 
+#include <mutex>
 #include <vector>
 
 #include "../../include/st_attn.h"
@@ -10,6 +11,7 @@
 // Natural-frame block CSR of one distinct (kind, offset): the exported, bit-exact contract.
 struct NatPlan {
     int32_t kind = 0, o = 0;
+    bool built = false;  // built on the first export (the kernels never read it)
     std::vector<int32_t> row_ptr, col_idx, mask_id;
     std::vector<uint32_t> masks;
     int32_t n_masks = 0;
@@ -20,7 +22,8 @@ struct st_layout {
     int64_t n = 0;
     int32_t l = 0, c = 0, block = 0;
     std::vector<int32_t> head_kind, head_off, head_plan;
-    std::vector<NatPlan> plans;
+    mutable std::vector<NatPlan> plans;
+    mutable std::mutex plans_mu;
 
     // execution plan (only when the kernels can run this layout)
     bool exec_ok = false;

@@ -132,7 +132,9 @@ ST_API st_status_t st_layout_head_kind(const st_layout_t *layout, int32_t head, 
  *   is allowed.  mask_id[e] is -1 when every pair of the block is allowed, else the index of
  *   its element mask: masks + mask_id * (block*block/32) u32 words, bit (r*block + cc) set iff
  *   (qb*block + r, kb*block + cc) is allowed, words little-endian.  Rows or columns past n are
- *   never set.  Identical masks are stored once per head kind. */
+ *   never set.  Identical masks are stored once per head kind.  The CSR of a head kind is built
+ *   on its first export (the kernels run the execution frames, not this view), so the first call
+ *   can take time at long n; ST_ERR_OOM if it does not fit in host memory. */
 ST_API st_status_t st_layout_export(const st_layout_t *layout, int32_t head, const int32_t **row_ptr,
                              const int32_t **col_idx, const int32_t **mask_id,
                              const uint32_t **masks, int32_t *n_qblk, int32_t *nnz,

@@ -57,6 +57,11 @@ def test_fwd_small_all_elements(w):
 
 
 BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
+# longer sequences (l about sqrt(n)), sampled rows: frames and work lists at 2^18 and 2^20 keys
+BIG += [Workload("s_n262144_l512_long", STRIDED, ALTERNATING, 262144, 512, 0, 1, 4),
+        Workload("s_merged_n262144_l512_long", STRIDED, MERGED, 262144, 512, 0, 1, 2),
+        Workload("s_n1048576_l1024_long", STRIDED, ALTERNATING, 1048576, 1024, 0, 1, 2),
+        Workload("f_n262144_l512_c128_long", FIXED, ALTERNATING, 262144, 512, 128, 1, 2)]
 
 # fp32 I/O: the n = 256 fp32 workload plus fixed and merged variants, every element compared
 FP32 = [WORKLOADS["strided_n256_l16_fp32"],
