@@ -57,7 +57,8 @@ struct Plan {
     static constexpr uint32_t STAGE = (SPLIT ? 3 : 2) * TB;     // K at +0, V at +TB, K_lo at +2TB
     static constexpr uint32_t OFF_P = OFF_STAGE + NST * STAGE;
     static constexpr uint32_t OFF_BAR = OFF_P + 2 * TB;
-    static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+    static constexpr uint32_t OFF_UNITS = OFF_BAR + 256;  // the claimed units' fields, NSCHED entries
+    static constexpr uint32_t SMEM_BYTES = OFF_UNITS + NSCHED * 96;
     static constexpr int MIN_BLOCKS = SPLIT ? 1 : CTAS_PER_SM;
 };
 
@@ -92,6 +93,7 @@ struct Unit {
     Part part;
     int32_t bh, nkt;
 };
+static_assert(sizeof(Unit) <= 96, "unit slot");
 
 __device__ __forceinline__ Unit load_unit(const FwdParams &p, int32_t u)
 {
@@ -104,16 +106,19 @@ __device__ __forceinline__ Unit load_unit(const FwdParams &p, int32_t u)
     return r;
 }
 
-// The j-th unit this CTA processes, as claimed by the producer: -1 when the list is exhausted,
-// -2 when the wait gave up.  Called by the MMA thread (warp_wide false) or by whole softmax warps.
-__device__ __forceinline__ int32_t next_unit(Bars *bars, int32_t j, bool warp_wide, volatile int32_t *abort,
-                                             int32_t *err)
+// The j-th unit this CTA processes, as claimed by the producer, with its fields copied out of
+// the shared slot j % NSCHED (which the producer fills; it may refill it once every consumer has
+// arrived): -1 when the list is exhausted, -2 when the wait gave up.  Called by the MMA thread
+// (warp_wide false) or by whole softmax warps.
+__device__ __forceinline__ int32_t next_unit(Bars *bars, const Unit *slots, int32_t j, bool warp_wide,
+                                             volatile int32_t *abort, int32_t *err, Unit &U)
 {
     const int s = j % NSCHED;
     bool ok = mbar_wait(&bars->sched_full[s], (j / NSCHED) & 1, abort, err);
     if (warp_wide) ok = __all_sync(0xffffffffu, ok);
     if (!ok) return -2;
     const int32_t u = *reinterpret_cast<volatile int32_t *>(&bars->sched[s]);
+    if (u >= 0) U = slots[s];
     if (warp_wide) __syncwarp();
     if (!warp_wide || (threadIdx.x & 31) == 0) mbar_arrive(&bars->sched_empty[s]);
     return u;
@@ -127,6 +132,7 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + L::OFF_BAR);
+    Unit *slots = reinterpret_cast<Unit *>(smem + L::OFF_UNITS);
     volatile int32_t *abort = &bars->abort;
     const int32_t nunits = p.nitems * p.batch;
 
@@ -210,9 +216,13 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 int32_t u = atomicAdd(p.sched, 1);
                 if (u >= nunits) u = -1;
                 bars->sched[s] = u;
+                Unit U;
+                if (u >= 0) {
+                    U = load_unit(p, u);
+                    slots[s] = U;
+                }
                 mbar_arrive(&bars->sched_full[s]);
                 if (u < 0) break;
-                const Unit U = load_unit(p, u);
                 if (U.nkt == 0) continue;
                 // the previous unit's S products must be done reading Q before it is replaced
                 if (kq > 0 && !mbar_wait(&bars->q_empty, (kq - 1) & 1, abort, p.err)) break;
@@ -276,9 +286,9 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
             int32_t T = 0, kq = 0;
             bool fail = false;
             for (int32_t j = 0; !fail; ++j) {
-                const int32_t u = next_unit(bars, j, false, abort, p.err);
+                Unit U;
+                const int32_t u = next_unit(bars, slots, j, false, abort, p.err, U);
                 if (u < 0) break;
-                const Unit U = load_unit(p, u);
                 if (U.nkt == 0) continue;
                 // Order per key tile: S(t+1) | PV_0(t) | PV_1(t).  S(t+1) overwrites S(t) as soon
                 // as both halves hold S(t) in registers (s_free), so the tensor pipe computes the
@@ -344,9 +354,9 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
         uint32_t v[64];
         int32_t T = 0, kq = 0;
         for (int32_t j = 0; ok; ++j) {
-            const int32_t u = next_unit(bars, j, true, abort, p.err);
+            Unit U;
+            const int32_t u = next_unit(bars, slots, j, true, abort, p.err, U);
             if (u < 0) break;
-            const Unit U = load_unit(p, u);
             int32_t lo_abs, hi_abs;
             const int32_t i = row_interval(p.g, U.part, U.w.tile, row, lo_abs, hi_abs);
             float m = -INFINITY, l = 0.f;
