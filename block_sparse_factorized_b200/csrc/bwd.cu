@@ -13,7 +13,7 @@
 //
 // The kernel is persistent (one CTA per SM) and claims items, longest first, from a global
 // counter.  K and V have two buffers, so the next item's loads and first S, dP products overlap
-// the current item's last tiles and its dK/dV epilogue.  Roles (576 threads):
+// the current item's last tiles and its dK/dV epilogue.  Roles (608 threads):
 //   warp 0      TMA: K and V of each item (KVS slots), Q and dO per query tile (2-stage ring)
 //   warp 1      MMA issuer: S = Q K^T and dP = dO V^T (TMEM, 128 x 128 fp32 each), then after
 //               the softmax warps wrote P and dS (bf16, SMEM): dV += P^T dO, dK += dS^T Q
@@ -24,6 +24,8 @@
 //               accumulator with a TMA reduce; at the end of an item one key row per thread:
 //               dK, dV columns 16g.. staged in SMEM for a TMA store (bf16), written row by row
 //               (fp32), or stored as the fp32 partial of a split key tile.
+//   warp 18     (bf16) the TMA stores of the staged dK, dV tiles, so that no softmax warp waits
+//               for them.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
 #include "tiles.cuh"
 
@@ -46,7 +48,8 @@ constexpr uint32_t OFF_ITEMS = OFF_BAR + 256;      // the claimed items' fields,
 constexpr uint32_t SMEM_BYTES = OFF_ITEMS + NSCHED * 96;
 constexpr int NWG = 4;                             // softmax warpgroups
 constexpr int NSM = 128 * NWG;                     // softmax threads
-constexpr int THREADS = 64 + NSM;
+constexpr int STORE_WARP = 2 + NSM / 32;           // the last warp
+constexpr int THREADS = 64 + NSM + 32;
 constexpr int CW = 128 / NWG;                      // score columns per warpgroup (32)
 constexpr int OW = 64 / NWG;                       // dQ / dK / dV columns per warpgroup (16)
 constexpr uint32_t TMEM_COLS = 512;
@@ -61,6 +64,7 @@ struct Bars {
     uint64_t stage_full, stage_free;  // bf16 dK/dV staged in the P area / its TMA store has read it
     uint64_t sched_full[NSCHED], sched_empty[NSCHED];
     int32_t sched[NSCHED];         // claimed item (index into items x batch), -1 = none left
+    int32_t store[4];              // staged tile: key frame, offset, key tile, batch-head (-1: end)
     uint32_t tmem_base;
     int32_t abort;
 };
@@ -299,6 +303,24 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             mma_commit(&bars->mma_idle);
             volatile int32_t never = 0;
             mbar_wait(&bars->mma_idle, 0, &never, p.err);
+        }
+    } else if (warp == STORE_WARP) {
+        // ---------------- dK, dV tile stores (bf16) ----------------
+        if (!F32 && lane == 0 && run) {
+            // the softmax warps stage one item's tiles at a time; the record says where they go
+            for (int32_t sf = 0;; ++sf) {
+                if (!mbar_wait(&bars->stage_full, sf & 1, abort, p.err)) break;
+                const volatile int32_t *r = bars->store;
+                const int32_t fr = r[0], o = r[1], tile = r[2], bh = r[3];
+                if (tile < 0) break;
+                if (*abort == 0) {
+                    store_tile(p.dk, fr, p.g, o, tile, bh, smem + OFF_P);
+                    store_tile(p.dv, fr, p.g, o, tile, bh, smem + OFF_P + TB);
+                    bulk_commit();
+                    bulk_wait_read_all();  // the next item's P stores may overwrite the staging
+                }
+                mbar_arrive(&bars->stage_free);
+            }
         }
     } else {
         // ------- P, dS, dQ drain, epilogue (warps 2..: warpgroup g owns score columns CW g..) -------
@@ -545,16 +567,13 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             if (staged) {
                 // the P area is free: dV of the last tile (its last reader) is done (dq_full)
                 fence_proxy_async_smem();
-                mbar_arrive(&bars->stage_full);
                 if (warp == 2 && lane == 0) {
-                    if (mbar_wait(&bars->stage_full, SF & 1, abort, p.err) && *abort == 0) {
-                        store_tile(p.dk, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, smem + OFF_P);
-                        store_tile(p.dv, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, smem + OFF_P + TB);
-                        bulk_commit();
-                        bulk_wait_read_all();  // the next item's P stores may overwrite the staging
-                    }
-                    mbar_arrive(&bars->stage_free);
+                    bars->store[0] = cur->part.kframe;
+                    bars->store[1] = cur->part.o;
+                    bars->store[2] = cur->w.tile;
+                    bars->store[3] = cur->bh;
                 }
+                mbar_arrive(&bars->stage_full);  // the store warp takes it from here
                 ++SF;
             }
             stage_pending = staged;
@@ -562,6 +581,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             J += nq;
         }
         if (lane == 0) bulk_wait_read_all();  // this warp's dQ reduces have read their staging
+        if (!F32 && ok && (!stage_pending || wait_all(&bars->stage_free, (SF - 1) & 1))) {
+            if (warp == 2 && lane == 0) bars->store[2] = -1;  // end of the store warp's loop
+            mbar_arrive(&bars->stage_full);
+        }
     }
     tc_fence_before();
     __syncthreads();
