@@ -36,6 +36,12 @@ SMALL = [
     Workload("f_merged_n1024_l128_c32", FIXED, MERGED, 1024, 128, 32, 1, 4),
     # long backward items: summary key tile 0 is read by all 64 query tiles
     Workload("f_n8192_l128_c32_long", FIXED, ALTERNATING, 8192, 128, 32, 1, 2),
+    # degenerate sets: c = l (pattern 2 reads every earlier key), c = 128 with three head-2
+    # offsets, fixed head 1 alone, odd batch and head counts
+    Workload("f_n512_l128_c128", FIXED, ALTERNATING, 512, 128, 128, 1, 2),
+    Workload("f_n1024_l256_c128_H6", FIXED, ALTERNATING, 1024, 256, 128, 1, 6),
+    Workload("f_single_a1_n512_l64", FIXED, SINGLE_A1, 512, 64, 16, 1, 2),
+    Workload("s_n384_l12_b3_H3", STRIDED, ALTERNATING, 384, 12, 0, 3, 3),
 ]
 
 

@@ -173,7 +173,8 @@ EXEC_SWEEP = [  # (family, mode, H, n, l, c) -- kernel-runnable layouts, every r
     (1, 1, 2, 512, 2, 0), (1, 2, 2, 256, 1, 0), (1, 1, 2, 256, 256, 0), (1, 2, 2, 768, 4, 0),
     (2, 1, 8, 512, 128, 32), (2, 2, 4, 512, 128, 32), (2, 1, 4, 1024, 256, 8),
     (2, 2, 4, 768, 64, 16), (2, 4, 4, 384, 128, 128), (1, 1, 2, 3072, 64, 0),
-    (1, 2, 2, 3072, 64, 0), (1, 1, 2, 32768, 256, 0),
+    (1, 2, 2, 3072, 64, 0), (1, 1, 2, 32768, 256, 0), (2, 1, 2, 512, 128, 128),
+    (2, 1, 6, 1024, 256, 128), (2, 3, 2, 512, 64, 16), (1, 1, 3, 384, 12, 0),
 ]
 
 
