@@ -378,13 +378,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             tmem_ld32(tS, sv);
             tmem_wait_ld();
             if (!(lo <= 0 && hi >= CW - 1)) {
-                const uint32_t span = static_cast<uint32_t>(hi - lo);
-                const bool none = hi < lo;
+                const uint32_t keep = interval_bits32(lo, hi);
 #pragma unroll
-                for (int e = 0; e < CW; ++e) {
-                    const bool keep = !none && static_cast<uint32_t>(e - lo) <= span;
-                    sv[e] = keep ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
-                }
+                for (int e = 0; e < CW; ++e) sv[e] = (keep & (1u << e)) ? sv[e] : 0xFF800000u;  // -inf: P = 0, dS = 0
             }
             {
                 const uint64_t sc2 = f32x2(sc, sc), nl2 = f32x2(nlse, nlse);

@@ -377,13 +377,11 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_free);  // the next S may overwrite this one
                 if (!(lo <= 0 && hi >= 63)) {  // boundary tile for this row: interval mask
-                    const uint32_t span = static_cast<uint32_t>(hi - lo);
-                    const bool none = hi < lo;
+                    const uint64_t keep = interval_bits64(lo, hi);
+                    const uint32_t k0 = static_cast<uint32_t>(keep), k1 = static_cast<uint32_t>(keep >> 32);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const bool keep = !none && static_cast<uint32_t>(c - lo) <= span;
-                        v[c] = keep ? v[c] : 0xFF800000u;  // -inf
-                    }
+                    for (int c = 0; c < 64; ++c)
+                        v[c] = ((c < 32 ? k0 : k1) & (1u << (c & 31))) ? v[c] : 0xFF800000u;  // -inf
                 }
                 const float m_tile = max64(v) * sc;
                 const float m_new = fmaxf(m, m_tile);
@@ -391,15 +389,21 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 const float m_use = grow ? m_new : m;
                 const float alpha = grow ? ex2(m - m_use) : 1.f;  // 0 when nothing was seen yet
                 const float nb = (m_use == -INFINITY) ? 0.f : -m_use;
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums
+                // p = exp2(s log2e / sqrt(d) - m), two columns per f32x2 instruction; two
+                // f32x2 partial sums
+                const uint64_t sc2 = f32x2(sc, sc), nb2 = f32x2(nb, nb);
+                uint64_t ps2[2] = {0ull, 0ull};
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    // p = exp2(s log2e / sqrt(d) - m)
-                    const float p0 = ex2(fmaf(__uint_as_float(v[c]), sc, nb));
-                    const float p1 = ex2(fmaf(__uint_as_float(v[c + 1]), sc, nb));
-                    ps[(c >> 1) & 3] += p0 + p1;
+                    float x0, x1;
+                    f32x2_split(fma2(f32x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2, nb2), x0, x1);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    ps2[(c >> 1) & 1] = add2(ps2[(c >> 1) & 1], f32x2(p0, p1));
                     v[c >> 1] = pack_bf16(p0, p1);
                 }
+                float ps[4];
+                f32x2_split(ps2[0], ps[0], ps[1]);
+                f32x2_split(ps2[1], ps[2], ps[3]);
                 // the previous PV of this half (possibly the previous unit's) must be done with
                 // P_h, and with O_h before a rescale
                 if (t > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[h], (t - 1) & 1, abort, p.err))) {

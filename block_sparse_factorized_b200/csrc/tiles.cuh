@@ -25,6 +25,25 @@ __device__ __forceinline__ float lg2(float x)
     return y;
 }
 
+// Columns lo..hi of a 64-column slice as a bit mask (bit c = column c allowed); lo and hi are
+// relative to the slice and may lie outside it; hi < lo is the empty interval.
+__device__ __forceinline__ uint64_t interval_bits64(int32_t lo, int32_t hi)
+{
+    if (hi < lo || hi < 0 || lo > 63) return 0ull;
+    const uint64_t up = hi >= 63 ? ~0ull : ((2ull << hi) - 1ull);
+    const uint64_t dn = lo <= 0 ? ~0ull : (~0ull << lo);
+    return up & dn;
+}
+
+// The same for a 32-column slice.
+__device__ __forceinline__ uint32_t interval_bits32(int32_t lo, int32_t hi)
+{
+    if (hi < lo || hi < 0 || lo > 31) return 0u;
+    const uint32_t up = hi >= 31 ? ~0u : ((2u << hi) - 1u);
+    const uint32_t dn = lo <= 0 ? ~0u : (~0u << lo);
+    return up & dn;
+}
+
 __device__ __forceinline__ const CUtensorMap *frame_map(const FrameMaps &m, int32_t fr)
 {
     return fr == FR_NAT ? &m.nat : (fr == FR_COL ? &m.col : &m.sum);
