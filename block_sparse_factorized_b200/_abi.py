@@ -51,7 +51,8 @@ class st_desc_t(ctypes.Structure):
 class st_layout_info_t(ctypes.Structure):
     _fields_ = [("fwd_items", ctypes.c_int64), ("exec_tiles", ctypes.c_int64),
                 ("bwd_items", ctypes.c_int64), ("allowed_pairs", ctypes.c_int64),
-                ("passes", ctypes.c_int32), ("split_passes", ctypes.c_int32)]
+                ("passes", ctypes.c_int32), ("split_passes", ctypes.c_int32),
+                ("dq_direct_heads", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -87,7 +88,7 @@ def load() -> ctypes.CDLL:
     lib.st_attn_fwd.argtypes = [P, P, P, P, P, P, P, sz, pp(st_desc_t), P]
     lib.st_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, sz, pp(st_desc_t), P]
     lib.st_attn_bwd_prepare.argtypes = [P, P, P, P, P, P, sz, pp(st_desc_t), P]
-    lib.st_attn_bwd_main.argtypes = [P, P, P, P, P, P, P, P, P, sz, pp(st_desc_t), P]
+    lib.st_attn_bwd_main.argtypes = [P, P, P, P, P, P, P, P, P, P, sz, pp(st_desc_t), P]
     lib.st_attn_bwd_finish.argtypes = [P, P, P, sz, pp(st_desc_t), P]
     lib.st_attn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, pp(st_desc_t), P]
     lib.st_attn_bwd_noalloc.restype = i32

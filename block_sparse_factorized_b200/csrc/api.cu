@@ -107,6 +107,19 @@ bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_
     return true;
 }
 
+// The dQ output in the natural frame with a 16-column, 32-row box: one warp's slice of a query
+// tile whose dQ the backward kernel stores directly (fp32: 64-byte swizzle, as the accumulator's
+// reduce map; bf16: 32-byte rows, 32-byte swizzle).
+bool make_map_dq_direct(CUtensorMap *m, const void *base, const st::Geom &g, int64_t BH, bool f32)
+{
+    const cuuint64_t row = 64 * (f32 ? 4 : 2), n = static_cast<cuuint64_t>(g.n);
+    const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+    const cuuint64_t str[2] = {row, n * row};
+    const cuuint32_t box[3] = {16, 32, 1};
+    return encode(m, base, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str,
+                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Frames {
@@ -293,27 +306,27 @@ st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t
     pre.dq_acc = ws.dq_acc;
     pre.dk = static_cast<uint16_t *>(dk);
     pre.dv = static_cast<uint16_t *>(dv);
-    pre.zero_fill = layout->d_zero_fill;
+    pre.head_flags = layout->d_head_flags;
     pre.counters = ws.counters;
     pre.ncounters = 2;
-    pre.rows = desc->batch * desc->heads * desc->n;
+    pre.bh = desc->batch * desc->heads;
     pre.n = static_cast<int32_t>(desc->n);
     pre.heads = static_cast<int32_t>(desc->heads);
     return st::launch_bwd_pre(pre, f32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
 st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
-                             const void *dO, const st_layout_t *layout, void *dk, void *dv,
+                             const void *dO, const st_layout_t *layout, void *dq, void *dk, void *dv,
                              void *workspace, size_t workspace_bytes, const st_desc_t *desc,
                              st_stream_t stream)
 {
-    if (!q || !k || !v || !lse || !dO || !dk || !dv) return ST_ERR_INVALID_ARG;
+    if (!q || !k || !v || !lse || !dO || !dq || !dk || !dv) return ST_ERR_INVALID_ARG;
     st_status_t cs = check_common(layout, desc);
     if (cs != ST_OK) return cs;
     BwdWs ws;
     if ((cs = bwd_workspace(desc, layout, workspace, workspace_bytes, ws)) != ST_OK) return cs;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lse) || !aligned16(dO) ||
-        !aligned16(dk) || !aligned16(dv))
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return ST_ERR_ALIGNMENT;
     const st_layout &L = *layout;
     const int64_t BH = desc->batch * desc->heads;
@@ -335,6 +348,7 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
         p.dk_f32 = static_cast<float *>(dk);
         p.dv_f32 = static_cast<float *>(dv);
     }
+    if (!make_map_dq_direct(&p.dq_direct, dq, L.geom, BH, f32)) return ST_ERR_CUDA;
     if (!make_maps_f32(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol)) return ST_ERR_CUDA;
     if (!f32 && (!make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum)))
         return ST_ERR_CUDA;
@@ -395,7 +409,10 @@ st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *worksp
     cv.dq_acc = ws.dq_acc;
     cv.dq = static_cast<uint16_t *>(dq);
     cv.dq_f32 = static_cast<float *>(dq);
-    cv.elems = desc->batch * desc->heads * desc->n * 64;
+    cv.head_flags = layout->d_head_flags;
+    cv.bh = desc->batch * desc->heads;
+    cv.n = static_cast<int32_t>(desc->n);
+    cv.heads = static_cast<int32_t>(desc->heads);
     return st::launch_dq_convert(cv, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
@@ -414,7 +431,7 @@ st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void 
         return ST_ERR_ALIGNMENT;
     if ((cs = st_attn_bwd_prepare(o, dO, layout, dk, dv, workspace, workspace_bytes, desc, stream)) != ST_OK)
         return cs;
-    if ((cs = st_attn_bwd_main(q, k, v, lse, dO, layout, dk, dv, workspace, workspace_bytes, desc,
+    if ((cs = st_attn_bwd_main(q, k, v, lse, dO, layout, dq, dk, dv, workspace, workspace_bytes, desc,
                                stream)) != ST_OK)
         return cs;
     return st_attn_bwd_finish(layout, dq, workspace, workspace_bytes, desc, stream);

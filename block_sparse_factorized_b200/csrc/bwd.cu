@@ -21,7 +21,8 @@
 //   warps 2..17 four warpgroups, one query row per thread, warpgroup g owning score columns
 //               32g..32g+31 (no row reduction is needed here: P comes from the saved lse):
 //               interval mask, P, dS; dQ columns 16g.. staged per warp and added to the fp32
-//               accumulator with a TMA reduce; at the end of an item one key row per thread:
+//               accumulator with a TMA reduce (or, where this item is the only one that reads
+//               the query tile, written to dQ directly); at the end of an item one key row per thread:
 //               dK, dV columns 16g.. staged in SMEM for a TMA store (bf16), written row by row
 //               (fp32), or stored as the fp32 partial of a split key tile.
 //   warp 18     (bf16) the TMA stores of the staged dK, dV tiles, so that no softmax warp waits
@@ -436,16 +437,31 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
             // per-warp staging (32 rows x 64 bytes, 64-byte swizzle): no cross-warp barrier
-            if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce has read it
+            if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce / store has read it
             __syncwarp();
+            const bool direct = cur->part.dq_direct != 0;  // the only contribution to these rows
+            if (!F32 && direct) {  // bf16 dQ itself: 32 rows x 32 bytes, 32-byte swizzle
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                st_shared_v4(sDQw + sw64_off(lane, q), dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
+                for (int q = 0; q < 2; ++q)
+                    st_shared_v4(sDQw + sw32_off(lane, q),
+                                 pack_bf16(__uint_as_float(dq[8 * q]), __uint_as_float(dq[8 * q + 1])),
+                                 pack_bf16(__uint_as_float(dq[8 * q + 2]), __uint_as_float(dq[8 * q + 3])),
+                                 pack_bf16(__uint_as_float(dq[8 * q + 4]), __uint_as_float(dq[8 * q + 5])),
+                                 pack_bf16(__uint_as_float(dq[8 * q + 6]), __uint_as_float(dq[8 * q + 7])));
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(sDQw + sw64_off(lane, q), dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                reduce_warp_f32(p.dq_red, cur->part.qframe, p.g, cur->w.begin + jj, cur->bh, OW * g, q4,
-                                smem + OFF_DQ + warp_slot);
+                if (direct)  // a natural-frame query part: a plain TMA store of the slice
+                    tma_store_3d(&p.dq_direct, smem + OFF_DQ + warp_slot, OW * g,
+                                 (cur->w.begin + jj) * TILE + 32 * q4, cur->bh);
+                else
+                    reduce_warp_f32(p.dq_red, cur->part.qframe, p.g, cur->w.begin + jj, cur->bh, OW * g, q4,
+                                    smem + OFF_DQ + warp_slot);
                 bulk_commit();
             }
         };

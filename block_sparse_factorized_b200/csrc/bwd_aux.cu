@@ -1,9 +1,9 @@
 // bwd_aux.cu -- the memory-bound passes around the backward kernel.
-//   bwd_pre:     D_i = dO_i . O_i (fp32), zero the fp32 dQ accumulator and the split key tiles'
-//                arrival counters, and zero dK/dV of heads whose keys are not all written by the
-//                main kernel (fixed pattern-2 heads read only summary positions; every other key
-//                gets no gradient).
-//   dq_convert:  dQ fp32 accumulator -> output dtype (round to nearest even).
+//   bwd_pre:     D_i = dO_i . O_i (fp32), zero the fp32 dQ accumulator (of heads whose dQ the main
+//                kernel does not write directly) and the work counters, and zero dK/dV of heads
+//                whose keys are not all written by the main kernel (fixed pattern-2 heads read
+//                only summary positions; every other key gets no gradient).
+//   dq_convert:  dQ fp32 accumulator -> output dtype (round to nearest even), same heads.
 //   split_finish: dK/dV of the backward's split key tiles from their chunks' fp32 partials.
 //   split:       fp32 tensor -> bf16 high part (round to nearest even) and optionally the bf16
 //                low part x - hi, the operands of the split-precision products of fp32 I/O.
@@ -14,64 +14,131 @@ namespace st {
 namespace {
 
 
+// Rows (of 64 values) each thread of the two passes below handles, their loads issued together:
+// with one 16- or 32-byte load per thread in flight the passes stop well short of HBM bandwidth.
+constexpr int UNROLL = 4;
+
+// Grid: x over chunks of 32 UNROLL rows of one batch-head, y over batch-heads (grid-stride both
+// ways), so that the per-head flags are read once per block.  Thread: one eighth (8 values) of
+// UNROLL rows 32 apart.
 template <bool F32>
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p)
+__global__ void __launch_bounds__(256, 4) bwd_pre_kernel(const PreParams p)
 {
-    for (int32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < p.ncounters; c += gridDim.x * blockDim.x)
-        p.counters[c] = 0;
-    const int64_t sub = threadIdx.x & 7;  // eighth of the 64-wide row
-    const int64_t nthr_rows = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 3);
-    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 3) + (threadIdx.x >> 3);
-         r < p.rows; r += nthr_rows) {
-        float s;
-        if (F32) {
-            const float4 *a = reinterpret_cast<const float4 *>(p.o_f32 + r * 64) + 2 * sub;
-            const float4 *b = reinterpret_cast<const float4 *>(p.dout_f32 + r * 64) + 2 * sub;
-            const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
-            s = a0.x * b0.x + a0.y * b0.y + a0.z * b0.z + a0.w * b0.w + a1.x * b1.x + a1.y * b1.y +
-                a1.z * b1.z + a1.w * b1.w;
-        } else {
-            const uint4 a = reinterpret_cast<const uint4 *>(p.o + r * 64)[sub];
-            const uint4 b = reinterpret_cast<const uint4 *>(p.dout + r * 64)[sub];
-            s = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
-                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
-                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
-        }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        if (sub == 0) p.delta[r] = s;
-        float4 *acc = reinterpret_cast<float4 *>(p.dq_acc + r * 64);
-        acc[2 * sub] = make_float4(0.f, 0.f, 0.f, 0.f);
-        acc[2 * sub + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const int32_t h = static_cast<int32_t>((r / p.n) % p.heads);
-        if (p.zero_fill[h]) {
+    constexpr int U = F32 ? 2 : UNROLL;  // fp32 rows: half as many per thread, in registers
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+        for (int32_t c = threadIdx.x; c < p.ncounters; c += blockDim.x) p.counters[c] = 0;
+    const int32_t sub = threadIdx.x & 7;  // eighth of the 64-wide row
+    const int32_t rpb = blockDim.x >> 3;
+    for (int64_t bh = blockIdx.y; bh < p.bh; bh += gridDim.y) {
+        const int32_t flags = p.head_flags[bh % p.heads];
+        const bool zero_dq = (flags & HEAD_DQ_DIRECT) == 0, zero_kv = (flags & HEAD_ZERO_FILL) != 0;
+        for (int32_t r0 = blockIdx.x * rpb * U + (threadIdx.x >> 3); r0 < p.n; r0 += gridDim.x * rpb * U) {
+            float s[U];
             if (F32) {
-                float4 *k4 = reinterpret_cast<float4 *>(p.dk_f32 + r * 64) + 2 * sub;
-                float4 *v4 = reinterpret_cast<float4 *>(p.dv_f32 + r * 64) + 2 * sub;
-                k4[0] = k4[1] = v4[0] = v4[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 a[U][2], b[U][2];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (r0 + u * rpb < p.n) {
+                        const int64_t r = bh * p.n + r0 + u * rpb;
+                        const float4 *pa = reinterpret_cast<const float4 *>(p.o_f32 + r * 64) + 2 * sub;
+                        const float4 *pb = reinterpret_cast<const float4 *>(p.dout_f32 + r * 64) + 2 * sub;
+                        a[u][0] = pa[0];
+                        a[u][1] = pa[1];
+                        b[u][0] = pb[0];
+                        b[u][1] = pb[1];
+                    }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    s[u] = 0.f;
+                    if (r0 + u * rpb < p.n)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            s[u] += a[u][h].x * b[u][h].x + a[u][h].y * b[u][h].y + a[u][h].z * b[u][h].z +
+                                    a[u][h].w * b[u][h].w;
+                }
             } else {
-                reinterpret_cast<uint4 *>(p.dk + r * 64)[sub] = make_uint4(0, 0, 0, 0);
-                reinterpret_cast<uint4 *>(p.dv + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+                uint4 a[U], b[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (r0 + u * rpb < p.n) {
+                        const int64_t r = bh * p.n + r0 + u * rpb;
+                        a[u] = reinterpret_cast<const uint4 *>(p.o + r * 64)[sub];
+                        b[u] = reinterpret_cast<const uint4 *>(p.dout + r * 64)[sub];
+                    }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    s[u] = (r0 + u * rpb < p.n)
+                               ? bf16_lo(a[u].x) * bf16_lo(b[u].x) + bf16_hi(a[u].x) * bf16_hi(b[u].x) +
+                                     bf16_lo(a[u].y) * bf16_lo(b[u].y) + bf16_hi(a[u].y) * bf16_hi(b[u].y) +
+                                     bf16_lo(a[u].z) * bf16_lo(b[u].z) + bf16_hi(a[u].z) * bf16_hi(b[u].z) +
+                                     bf16_lo(a[u].w) * bf16_lo(b[u].w) + bf16_hi(a[u].w) * bf16_hi(b[u].w)
+                               : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {  // the 8 threads of a row sum their eighths
+                s[u] += __shfl_xor_sync(0xffffffffu, s[u], 1);
+                s[u] += __shfl_xor_sync(0xffffffffu, s[u], 2);
+                s[u] += __shfl_xor_sync(0xffffffffu, s[u], 4);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (r0 + u * rpb >= p.n) continue;
+                const int64_t r = bh * p.n + r0 + u * rpb;
+                if (sub == 0) p.delta[r] = s[u];
+                if (zero_dq) {
+                    float4 *acc = reinterpret_cast<float4 *>(p.dq_acc + r * 64);
+                    acc[2 * sub] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    acc[2 * sub + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                if (zero_kv) {
+                    if (F32) {
+                        float4 *k4 = reinterpret_cast<float4 *>(p.dk_f32 + r * 64) + 2 * sub;
+                        float4 *v4 = reinterpret_cast<float4 *>(p.dv_f32 + r * 64) + 2 * sub;
+                        k4[0] = k4[1] = v4[0] = v4[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    } else {
+                        reinterpret_cast<uint4 *>(p.dk + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+                        reinterpret_cast<uint4 *>(p.dv + r * 64)[sub] = make_uint4(0, 0, 0, 0);
+                    }
+                }
             }
         }
     }
 }
 
+// Same grid as bwd_pre_kernel; a thread converts UNROLL groups of 8 consecutive values, 256
+// groups apart.
 template <bool F32>
-__global__ void __launch_bounds__(256) dq_convert_kernel(const ConvParams p)
+__global__ void __launch_bounds__(256, 4) dq_convert_kernel(const ConvParams p)
 {
-    const int64_t n8 = p.elems / 8;
-    for (int64_t a = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; a < n8;
-         a += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const float4 x = reinterpret_cast<const float4 *>(p.dq_acc)[2 * a];
-        const float4 y = reinterpret_cast<const float4 *>(p.dq_acc)[2 * a + 1];
-        if (F32) {
-            reinterpret_cast<float4 *>(p.dq_f32)[2 * a] = x;
-            reinterpret_cast<float4 *>(p.dq_f32)[2 * a + 1] = y;
-        } else {
-            reinterpret_cast<uint4 *>(p.dq)[a] = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w),
-                                                            pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+    const int64_t n8 = static_cast<int64_t>(p.n) * 8;  // 8-value groups per batch-head
+    for (int64_t bh = blockIdx.y; bh < p.bh; bh += gridDim.y) {
+        if (p.head_flags[bh % p.heads] & HEAD_DQ_DIRECT) continue;  // written by the main kernel
+        const float4 *src = reinterpret_cast<const float4 *>(p.dq_acc) + bh * n8 * 2;
+        for (int64_t a0 = static_cast<int64_t>(blockIdx.x) * blockDim.x * UNROLL + threadIdx.x; a0 < n8;
+             a0 += static_cast<int64_t>(gridDim.x) * blockDim.x * UNROLL) {
+            float4 x[UNROLL], y[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int64_t a = a0 + u * static_cast<int64_t>(blockDim.x);
+                if (a < n8) {
+                    x[u] = src[2 * a];
+                    y[u] = src[2 * a + 1];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int64_t a = a0 + u * static_cast<int64_t>(blockDim.x);
+                if (a >= n8) continue;
+                const int64_t e = bh * n8 + a;
+                if (F32) {
+                    reinterpret_cast<float4 *>(p.dq_f32)[2 * e] = x[u];
+                    reinterpret_cast<float4 *>(p.dq_f32)[2 * e + 1] = y[u];
+                } else {
+                    reinterpret_cast<uint4 *>(p.dq)[e] =
+                        make_uint4(pack_bf16(x[u].x, x[u].y), pack_bf16(x[u].z, x[u].w), pack_bf16(y[u].x, y[u].y),
+                                   pack_bf16(y[u].z, y[u].w));
+                }
+            }
         }
     }
 }
@@ -193,23 +260,31 @@ int blocks_for(int64_t work_units)
     return static_cast<int>(work_units < cap ? (work_units > 0 ? work_units : 1) : cap);
 }
 
+// x: chunks of one batch-head's rows (at most 4096 blocks), y: batch-heads (at most 65535)
+static dim3 head_grid(int64_t chunks, int64_t bh)
+{
+    const int64_t x = chunks < 1 ? 1 : (chunks > 4096 ? 4096 : chunks);
+    const int64_t y = bh < 1 ? 1 : (bh > 65535 ? 65535 : bh);
+    return dim3(static_cast<unsigned>(x), static_cast<unsigned>(y));
+}
+
 cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s)
 {
-    const int blocks = blocks_for((p.rows + 31) / 32);
+    const dim3 grid = head_grid((p.n + 32 * UNROLL - 1) / (32 * UNROLL), p.bh);
     if (f32)
-        bwd_pre_kernel<true><<<blocks, 256, 0, s>>>(p);
+        bwd_pre_kernel<true><<<grid, 256, 0, s>>>(p);
     else
-        bwd_pre_kernel<false><<<blocks, 256, 0, s>>>(p);
+        bwd_pre_kernel<false><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s)
 {
-    const int blocks = blocks_for((p.elems / 8 + 255) / 256);
+    const dim3 grid = head_grid((static_cast<int64_t>(p.n) * 8 + 256 * UNROLL - 1) / (256 * UNROLL), p.bh);
     if (f32)
-        dq_convert_kernel<true><<<blocks, 256, 0, s>>>(p);
+        dq_convert_kernel<true><<<grid, 256, 0, s>>>(p);
     else
-        dq_convert_kernel<false><<<blocks, 256, 0, s>>>(p);
+        dq_convert_kernel<false><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

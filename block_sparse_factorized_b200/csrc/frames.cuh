@@ -86,8 +86,14 @@ struct Part {
     int32_t lo_off, hi_off;
     int32_t merge;         // 1: second pass, merges into what the first pass wrote
     int32_t nq, nk;        // tiles in the query / key frame
-    int32_t pad[2];
+    int32_t dq_direct;     // 1: each query tile of the head is read by exactly one backward item
+                           // (of any pass), so that item writes its dQ rows directly
+    int32_t pad;
 };
+
+// Per-head flags of the backward pass.
+constexpr int32_t HEAD_ZERO_FILL = 1;   // some key is written by no pass-0 item: dK, dV zeroed first
+constexpr int32_t HEAD_DQ_DIRECT = 2;   // dQ written by the main kernel (see Part::dq_direct)
 
 struct WorkItem {          // fwd: tile = query tile, [begin,end) key tiles; bwd: the converse
     int32_t part, tile, begin, end;

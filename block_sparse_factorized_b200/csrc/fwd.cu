@@ -593,7 +593,7 @@ cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t s)
 
 cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s)
 {
-    return split ? launch_fwd_t<true>(p, s) : launch_fwd_t<false>(p, s);
+    return split ? launch_fwd_t<true>(p, s) : launch_fwd_bf16(p, s);
 }
 
 }  // namespace st

@@ -36,8 +36,11 @@ struct FwdParams {
 struct BwdParams {
     FrameMaps q, k, v, dout;
     FrameMaps dk, dv;            // bf16 I/O: dK, dV tile stores (sum used for compacted keys)
-    FrameMaps dq_red;            // fp32 dQ accumulator in the query frames, box 32 columns wide
-                                 // (reduce-add target; nat and col only)
+    FrameMaps dq_red;            // fp32 dQ accumulator in the query frames, box 16 columns by
+                                 // 32 rows (reduce-add target; nat and col only)
+    CUtensorMap dq_direct;       // dQ output (natural frame), box 16 columns by 32 rows: one
+                                 // warp's slice of a dq_direct part (fp32: 64-byte swizzle,
+                                 // bf16: 32-byte swizzle)
     const Part *parts;
     const WorkItem *items;
     int32_t nitems, batch, heads;
@@ -59,12 +62,12 @@ struct PreParams {
     const float *o_f32, *dout_f32;  // fp32 I/O instead of o, dout
     float *dk_f32, *dv_f32;         // fp32 I/O instead of dk, dv
     float *delta;                // [B*H, n]
-    float *dq_acc;               // [B*H, n, 64] zeroed here
-    uint16_t *dk, *dv;           // zero-filled for heads flagged in zero_fill
-    const int32_t *zero_fill;    // [H]
+    float *dq_acc;               // [B*H, n, 64] zeroed here (heads without HEAD_DQ_DIRECT)
+    uint16_t *dk, *dv;           // zero-filled for heads flagged HEAD_ZERO_FILL
+    const int32_t *head_flags;   // [H]
     int32_t *counters;           // zeroed here
     int32_t ncounters;
-    int64_t rows;                // B*H*n
+    int64_t bh;                  // B*H
     int32_t n, heads;
 };
 
@@ -72,7 +75,9 @@ struct ConvParams {
     const float *dq_acc;
     uint16_t *dq;
     float *dq_f32;               // fp32 I/O: plain copy instead of rounding to bf16
-    int64_t elems;
+    const int32_t *head_flags;   // [H]: heads with HEAD_DQ_DIRECT are skipped
+    int64_t bh;                  // B*H
+    int32_t n, heads;
 };
 
 // dK/dV of split key tiles: sum of the chunks' fp32 partials in chunk order, plus the first
@@ -95,6 +100,7 @@ struct SplitParams {
 };
 
 cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s);
+cudaError_t launch_fwd_bf16(const FwdParams &p, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s);

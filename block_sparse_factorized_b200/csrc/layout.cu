@@ -276,7 +276,7 @@ st_status_t build_exec(st_layout &L)
                 static_cast<int32_t>(a * 1000000000 + k);
         }
     // heads whose pass-0 backward leaves some key unwritten need a zero fill first
-    L.head_zero_fill.assign(static_cast<size_t>(H), 0);
+    L.head_flags.assign(static_cast<size_t>(H), 0);
     std::vector<uint8_t> cov(static_cast<size_t>(n));
     for (int32_t h = 0; h < H; ++h) {
         std::fill(cov.begin(), cov.end(), 0);
@@ -289,7 +289,27 @@ st_status_t build_exec(st_layout &L)
             }
         }
         for (int64_t j = 0; j < n; ++j)
-            if (!cov[j]) { L.head_zero_fill[h] = 1; break; }
+            if (!cov[j]) { L.head_flags[h] |= st::HEAD_ZERO_FILL; break; }
+    }
+    // heads whose every (natural-frame) query tile is read by exactly one backward item, of
+    // either pass: that item's dQ tile is the whole gradient of its rows and is written directly,
+    // with no fp32 accumulation
+    std::vector<int32_t> qcnt(static_cast<size_t>(n / st::TILE));
+    for (int32_t h = 0; h < H; ++h) {
+        bool nat = true;
+        for (const auto &p : L.parts)
+            if (p.head == h && p.qframe != st::FR_NAT) nat = false;
+        if (!nat) continue;
+        std::fill(qcnt.begin(), qcnt.end(), 0);
+        for (int a = 0; a < 2; ++a)
+            for (const auto &w : L.bwd_items[a])
+                if (L.parts[w.part].head == h)
+                    for (int32_t qt = w.begin; qt < w.end; ++qt) ++qcnt[qt];
+        if (std::all_of(qcnt.begin(), qcnt.end(), [](int32_t x) { return x == 1; })) {
+            L.head_flags[h] |= st::HEAD_DQ_DIRECT;
+            for (auto &p : L.parts)
+                if (p.head == h) p.dq_direct = 1;
+        }
     }
     return ST_OK;
 }
@@ -373,7 +393,7 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
     const size_t nf1 = L->fwd_items[1].size() * sizeof(st::WorkItem);
     const size_t nb0 = L->bwd_items[0].size() * sizeof(st::WorkItem);
     const size_t nb1 = L->bwd_items[1].size() * sizeof(st::WorkItem);
-    const size_t nz = L->head_zero_fill.size() * sizeof(int32_t);
+    const size_t nz = L->head_flags.size() * sizeof(int32_t);
     const size_t ns0 = L->bwd_split_recs[0].size() * sizeof(st::SplitRec);
     const size_t ns1 = L->bwd_split_recs[1].size() * sizeof(st::SplitRec);
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
@@ -390,7 +410,7 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
         L->d_fwd[1] = reinterpret_cast<st::WorkItem *>(b + off_f1);
         L->d_bwd[0] = reinterpret_cast<st::WorkItem *>(b + off_b0);
         L->d_bwd[1] = reinterpret_cast<st::WorkItem *>(b + off_b1);
-        L->d_zero_fill = reinterpret_cast<int32_t *>(b + off_z);
+        L->d_head_flags = reinterpret_cast<int32_t *>(b + off_z);
         L->d_split[0] = reinterpret_cast<st::SplitRec *>(b + off_s0);
         L->d_split[1] = reinterpret_cast<st::SplitRec *>(b + off_s1);
         L->d_err = reinterpret_cast<int32_t *>(b + off_e);
@@ -400,7 +420,7 @@ st_status_t st_layout_upload(st_layout_t *L, st_stream_t stream)
     };
     if (!cp(L->d_parts, L->parts.data(), np) || !cp(L->d_fwd[0], L->fwd_items[0].data(), nf0) ||
         !cp(L->d_fwd[1], L->fwd_items[1].data(), nf1) || !cp(L->d_bwd[0], L->bwd_items[0].data(), nb0) ||
-        !cp(L->d_bwd[1], L->bwd_items[1].data(), nb1) || !cp(L->d_zero_fill, L->head_zero_fill.data(), nz) ||
+        !cp(L->d_bwd[1], L->bwd_items[1].data(), nb1) || !cp(L->d_head_flags, L->head_flags.data(), nz) ||
         !cp(L->d_split[0], L->bwd_split_recs[0].data(), ns0) || !cp(L->d_split[1], L->bwd_split_recs[1].data(), ns1))
         return ST_ERR_CUDA;
     L->uploaded = true;
@@ -451,6 +471,8 @@ st_status_t st_layout_info(const st_layout_t *L, st_layout_info_t *info)
     info->allowed_pairs = L->allowed_pairs;
     info->passes = L->passes;
     info->split_passes = (L->bwd_split_recs[0].empty() ? 0 : 1) + (L->bwd_split_recs[1].empty() ? 0 : 1);
+    for (const int32_t f : L->head_flags)
+        if (f & st::HEAD_DQ_DIRECT) ++info->dq_direct_heads;
     return ST_OK;
 }
 

@@ -29,7 +29,7 @@ struct st_layout {
     bool exec_ok = false;
     st::Geom geom{};
     std::vector<st::Part> parts;
-    std::vector<int32_t> head_zero_fill;   // 1: some key of this head is read by no pass-0 part
+    std::vector<int32_t> head_flags;       // HEAD_ZERO_FILL | HEAD_DQ_DIRECT per head
     std::vector<st::WorkItem> fwd_items[2], bwd_items[2];
     int32_t passes = 1;
     int32_t bwd_slots = 0, bwd_splits = 0;  // partial-sum slots and split key tiles (bwd)
@@ -44,7 +44,7 @@ struct st_layout {
     st::Part *d_parts = nullptr;
     st::WorkItem *d_fwd[2] = {nullptr, nullptr};
     st::WorkItem *d_bwd[2] = {nullptr, nullptr};
-    int32_t *d_zero_fill = nullptr;
+    int32_t *d_head_flags = nullptr;
     st::SplitRec *d_split[2] = {nullptr, nullptr};
     int32_t *d_err = nullptr;
 };

@@ -214,6 +214,20 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// D (TMEM, fp32) (+)= A B with A read from TMEM: lane m holds row m of A, 16-bit elements packed
+// two per 32-bit column along K (the lower-indexed element in the low half), so one K = 16 step
+// spans 8 columns.  B from shared memory as for mma_bf16_ss.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
@@ -348,6 +362,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
+}
+
+// Byte offset of logical 16-byte chunk `ch` (0..1) of row `r` in a 32-byte-swizzled tile
+// (32-byte rows; chunk index XOR bit 2 of the row).
+__device__ __forceinline__ uint32_t sw32_off(uint32_t r, uint32_t ch)
+{
+    return r * 32u + ((ch ^ ((r >> 2) & 1u)) << 4);
 }
 
 // Byte offset of logical 16-byte chunk `ch` (0..3) of row `r` in a 64-byte-swizzled tile

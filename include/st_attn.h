@@ -149,6 +149,9 @@ typedef struct {
     int32_t passes;         /* 1, or 2 for merged strided heads (band part, then grid part) */
     int32_t split_passes;   /* passes with a key tile whose query run is split over several CTAs
                                (each adds one short summing launch to the backward pass) */
+    int32_t dq_direct_heads; /* heads whose every query tile is read by one backward item: their
+                                dQ is written by st_attn_bwd_main, not accumulated */
+    int32_t reserved;       /* 0 */
 } st_layout_info_t;
 ST_API st_status_t st_layout_info(const st_layout_t *layout, st_layout_info_t *info);
 
@@ -191,15 +194,18 @@ ST_API st_status_t st_attn_bwd(const void *q, const void *k, const void *v, cons
  * with the same workspace) to time or overlap them:
  *   st_attn_bwd_prepare  D_i = dO_i . O_i into the workspace, zero the fp32 dQ accumulator, and
  *                        zero dK/dV of heads whose keys are not all written by the main phase
- *   st_attn_bwd_main     the recomputing tcgen05 kernel: dK, dV written, dQ accumulated
- *   st_attn_bwd_finish   dQ accumulator -> dq (output dtype)
+ *   st_attn_bwd_main     the recomputing tcgen05 kernel: dK, dV written, dQ accumulated -- or,
+ *                        for a head whose every query tile is read by a single key tile (the
+ *                        fixed pattern's same-block head with l = 128), written to dq directly
+ *   st_attn_bwd_finish   dQ accumulator -> dq (output dtype) for the other heads
  * Arguments as for st_attn_bwd; errors as for st_attn_bwd. */
 ST_API st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t *layout,
                                        void *dk, void *dv, void *workspace,
                                        size_t workspace_bytes, const st_desc_t *desc,
                                        st_stream_t stream);
 ST_API st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
-                                    const void *dO, const st_layout_t *layout, void *dk, void *dv,
+                                    const void *dO, const st_layout_t *layout, void *dq, void *dk,
+                                    void *dv,
                                     void *workspace, size_t workspace_bytes,
                                     const st_desc_t *desc, st_stream_t stream);
 ST_API st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *workspace,

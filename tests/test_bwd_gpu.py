@@ -9,6 +9,8 @@ import numpy as np
 import pytest
 import torch
 
+import ctypes
+
 import oracle
 from parity import check_grads, cuda_inputs, problem_of, rel_l2, sample_rows, to64
 from test_fwd_gpu import FP32, SMALL
@@ -115,3 +117,47 @@ def test_autograd_wrapper():
     out.backward(dod)
     ref = problem_of(w).bwd(to64(q), to64(k), to64(v), to64(do))
     check_grads((to64(qg.grad), to64(kg.grad), to64(vg.grad)), ref, "autograd")
+
+
+@pytest.mark.parametrize("w", [Workload("f_n512_l128_c32_b2", FIXED, ALTERNATING, 512, 128, 32, 2, 2),
+                               Workload("f_n1024_l128_c32_H4", FIXED, ALTERNATING, 1024, 128, 32, 1, 4)],
+                         ids=lambda w: w.name)
+def test_bwd_phases_and_direct_dq(w):
+    """st_attn_bwd_prepare / _main / _finish called one by one give st_attn_bwd's results, and
+    the dQ of heads whose query tiles are each read by a single backward item (written by the main
+    kernel, no accumulation) is bitwise repeatable."""
+    from block_sparse_factorized_b200 import _abi
+    (qd, kd, vd, dod), (q, k, v, do) = cuda_inputs(w)
+    lay, o, lse, dq1, dk1, dv1 = run(w, qd, kd, vd, dod)
+    lib = _abi.load()
+    desc = bsf._desc(qd)
+    nbytes = int(lib.st_attn_bwd_workspace_bytes(ctypes.byref(desc), lay.handle))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=qd.device)
+    dq2, dk2, dv2 = (torch.full_like(qd, float("nan")) for _ in range(3))
+    P = ctypes.c_void_p
+    ptr = lambda t: P(t.data_ptr())  # noqa: E731
+    sp = P(torch.cuda.current_stream().cuda_stream)
+    _abi.check(lib.st_attn_bwd_prepare(ptr(o), ptr(dod), lay.handle, ptr(dk2), ptr(dv2), ptr(ws), nbytes,
+                                       ctypes.byref(desc), sp), "st_attn_bwd_prepare")
+    _abi.check(lib.st_attn_bwd_main(ptr(qd), ptr(kd), ptr(vd), ptr(lse), ptr(dod), lay.handle, ptr(dq2),
+                                    ptr(dk2), ptr(dv2), ptr(ws), nbytes, ctypes.byref(desc), sp),
+               "st_attn_bwd_main")
+    _abi.check(lib.st_attn_bwd_finish(lay.handle, ptr(dq2), ptr(ws), nbytes, ctypes.byref(desc), sp),
+               "st_attn_bwd_finish")
+    torch.cuda.synchronize()
+    lay.check()
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    info = lay.info()
+    kinds, _ = oracle.head_kinds(w.family, w.head_mode, w.heads, w.l, w.c, w.offset_step)
+    # which heads are direct: the same-block heads (one key tile per query tile at l = 128), and
+    # the summary heads when every summary key fits one compacted tile (n / l * c <= 128)
+    direct = [h for h in range(w.heads)
+              if int(kinds[h]) == oracle.FA1 or (w.n // w.l) * w.c <= 128]
+    assert info["dq_direct_heads"] == len(direct)
+    for h in range(w.heads):
+        if h in direct:
+            assert torch.equal(dq1[:, h], dq2[:, h]), h
+        else:
+            assert rel_l2(to64(dq1[:, h]), to64(dq2[:, h])) < 1e-3, h
+    ref = problem_of(w).bwd(to64(q), to64(k), to64(v), to64(do))
+    check_grads((to64(dq2), to64(dk2), to64(dv2)), ref, w.name)

@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 
 import oracle
-from workloads import WORKLOADS
+from workloads import ALTERNATING, FIXED, MERGED, WORKLOADS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -214,3 +214,24 @@ def test_exec_tile_counts():
         for kd, off in zip(*kinds[0]):
             total += int(oracle.set_counts(int(kd), wl.n, wl.l, wl.c, int(off)).sum())
         assert info["allowed_pairs"] == total, name
+
+
+def test_dq_direct_heads():
+    """Heads whose every query tile is read by exactly one backward item (summed over passes)
+    have their dQ written by the main kernel instead of accumulated."""
+    w = WORKLOADS["fixed_n12288_l128_c32"]
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c)
+    assert lay.info()["dq_direct_heads"] == 4   # the four same-block heads (l = 128 = one tile)
+    for name in ("strided_n12288_l128", "strided_merged_n12288_l128", "strided_n65536_l256",
+                 "strided_merged_n3072_l64"):
+        wl = WORKLOADS[name]
+        assert bsf.Layout(wl.family, wl.head_mode, wl.heads, wl.n, wl.l, wl.c).info()["dq_direct_heads"] == 0
+    # n = 512, l = 128, c = 32: the summary keys of all four blocks fill one compacted tile, so the
+    # summary head is direct too
+    assert bsf.Layout(FIXED, ALTERNATING, 2, 512, 128, 32).info()["dq_direct_heads"] == 2
+    # l = 256: odd query tiles read two key tiles of their block; in the summary head, query tile 0
+    # (rows 0-127 of block 0, all before the block's summary run) is read by no item, so its dQ
+    # rows are left to the accumulator's zeros
+    assert bsf.Layout(FIXED, ALTERNATING, 2, 1024, 256, 32).info()["dq_direct_heads"] == 0
+    # merged fixed heads: same-block pass plus the earlier blocks' summaries (two items per tile)
+    assert bsf.Layout(FIXED, MERGED, 2, 1024, 128, 32).info()["dq_direct_heads"] == 0
