@@ -1,4 +1,8 @@
-// fwd.cu -- fused forward pass of factorized sparse attention on sm_100a.
+// fwd.cu -- fused forward pass of factorized sparse attention on sm_100a, fp32 I/O.
+//
+// fp32 inputs are split into bf16 high and low parts (hi = bf16(x), lo = bf16(x - hi)) and the
+// scores take three products, S = Q_hi K_hi^T + Q_hi K_lo^T + Q_lo K_hi^T, all accumulated in
+// fp32 in TMEM; P V runs on bf16 P and V_hi.  (bf16 I/O runs the kernel in fwd_bf16.cu.)
 //
 // Each work unit is one 128-row query tile of one part of one (batch, head) over the contiguous
 // run of 128-key tiles its work item lists ("Sparse Transformers（稀疏 Transformer）深度解读报告"
@@ -16,10 +20,11 @@
 //   M = max(m_0, m_1), L = sum_h 2^(m_h - M) l_h, O = sum_h 2^(m_h - M) O_h / L, lse = M + log2 L
 // (log2 units).  No per-tile exchange between the warpgroups is needed.
 //
-// The kernel is persistent: two CTAs per SM claim units from the longest-first list through a
-// global counter (greedy list scheduling).  Barrier phases run on across units, so the next
-// unit's Q load and first S product overlap the current unit's last softmax and epilogue.  Roles (320 threads):
-//   warp 0       TMA producer: Q (and its low part for split precision), K and V tiles in NST-slot
+// The kernel is persistent: one CTA per SM (the high and low parts fill the shared memory of two)
+// claims units from the longest-first list through a global counter (greedy list scheduling).
+// Barrier phases run on across units, so the next unit's Q load and first S product overlap the
+// current unit's last softmax and epilogue.  Roles (320 threads):
+//   warp 0       TMA producer: Q and its low part, K (with its low part) and V tiles in NST-slot
 //                rings with separate barriers
 //   warp 1       MMA issuer (one thread): S = Q K^T into TMEM (128 x 128 fp32), issued for the
 //                next key tile as soon as the softmax warps hold the current S in registers;
@@ -30,7 +35,7 @@
 //                only when the row max grew by more than 2^8 (otherwise the stale max is kept:
 //                numerator and denominator use the same max, so the result is unchanged);
 //                then the unit's epilogue: combine the halves (each warpgroup writes 32 of the 64
-//                output columns straight to global memory), a merge part folds in the first
+//                fp32 output columns straight to global memory), a merge part folds in the first
 //                pass's (O, lse).
 #include "tiles.cuh"
 
@@ -41,25 +46,22 @@ constexpr int NST = 2;                         // K/V ring depth
 constexpr int NSCHED = 4;                      // claimed-unit ring depth
 constexpr uint32_t TB = TILE_BYTES;            // one 128 x 64 bf16 tile, 16 KB
 constexpr int THREADS = 320;
-constexpr int CTAS_PER_SM = 2;
 constexpr uint32_t TMEM_COLS = 256;            // S: 0..127, O_0: 128..191, O_1: 192..255
 constexpr float RESCALE_LOG2 = 8.0f;           // keep a stale max while it is within 2^8
 
-// Shared-memory plan.  SPLIT (fp32 I/O) adds the low bf16 parts of Q and of each K tile.
+// Shared-memory plan: the bf16 high and low parts of Q and of each K tile.
 //   Q [, Q_lo] | NST x (K, V [, K_lo]) | P (two 128 x 64 halves: keys 0-63, 64-127) | barriers
 // The P area doubles as the (m, l) exchange of the epilogue.
-template <bool SPLIT>
 struct Plan {
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_QL = TB;
-    static constexpr uint32_t QBYTES = (SPLIT ? 2 : 1) * TB;
+    static constexpr uint32_t QBYTES = 2 * TB;
     static constexpr uint32_t OFF_STAGE = QBYTES;
-    static constexpr uint32_t STAGE = (SPLIT ? 3 : 2) * TB;     // K at +0, V at +TB, K_lo at +2TB
+    static constexpr uint32_t STAGE = 3 * TB;                   // K at +0, V at +TB, K_lo at +2TB
     static constexpr uint32_t OFF_P = OFF_STAGE + NST * STAGE;
     static constexpr uint32_t OFF_BAR = OFF_P + 2 * TB;
     static constexpr uint32_t OFF_UNITS = OFF_BAR + 256;  // the claimed units' fields, NSCHED entries
     static constexpr uint32_t SMEM_BYTES = OFF_UNITS + NSCHED * 96;
-    static constexpr int MIN_BLOCKS = SPLIT ? 1 : CTAS_PER_SM;
 };
 
 struct Bars {
@@ -124,11 +126,10 @@ __device__ __forceinline__ int32_t next_unit(Bars *bars, const Unit *slots, int3
     return u;
 }
 
-template <bool SPLIT>
-__global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
-    fwd_kernel(const __grid_constant__ FwdParams p)
+__global__ void __launch_bounds__(THREADS, 1)
+    fwd_split_kernel(const __grid_constant__ FwdParams p)
 {
-    using L = Plan<SPLIT>;
+    using L = Plan;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + L::OFF_BAR);
@@ -191,9 +192,9 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 const int s = TK % NST;
                 if (TK >= NST && !mbar_wait(&bars->k_empty[s], ((TK / NST) - 1) & 1, abort, p.err)) return false;
                 uint8_t *stage = smem + L::OFF_STAGE + s * L::STAGE;
-                mbar_arrive_expect_tx(&bars->k_full[s], (SPLIT ? 2 : 1) * TB);
+                mbar_arrive_expect_tx(&bars->k_full[s], 2 * TB);
                 load_tile(p.k, U.part.kframe, p.g, U.part.o, tile, U.bh, stage, &bars->k_full[s]);
-                if (SPLIT) load_tile(p.kl, U.part.kframe, p.g, U.part.o, tile, U.bh, stage + 2 * TB, &bars->k_full[s]);
+                load_tile(p.kl, U.part.kframe, p.g, U.part.o, tile, U.bh, stage + 2 * TB, &bars->k_full[s]);
                 ++TK;
                 return true;
             };
@@ -229,8 +230,7 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 ++kq;
                 mbar_arrive_expect_tx(&bars->q_full, L::QBYTES);
                 load_tile(p.q, U.part.qframe, p.g, U.part.o, U.w.tile, U.bh, smem + L::OFF_Q, &bars->q_full);
-                if (SPLIT)
-                    load_tile(p.ql, U.part.qframe, p.g, U.part.o, U.w.tile, U.bh, smem + L::OFF_QL, &bars->q_full);
+                load_tile(p.ql, U.part.qframe, p.g, U.part.o, U.w.tile, U.bh, smem + L::OFF_QL, &bars->q_full);
                 fail = !load_k(U, U.w.begin);
                 for (int it = 0; !fail && it < U.nkt; ++it)
                     fail = (it + 1 < U.nkt && !load_k(U, U.w.begin + it + 1)) || !load_v(U, U.w.begin + it);
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
                 for (int k = 0; k < 4; ++k)
                     mma_bf16_ss(tS, desc_sw128(sQ + 32 * k, 16, 1024),
                                 desc_sw128(sK + 32 * k, 16, 1024), idS, k > 0 ? 1u : 0u);
-                if (SPLIT) {
+                {
                     const uint32_t sQl = smem_u32(smem + L::OFF_QL), sKl = sK + 2 * TB;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -506,45 +506,22 @@ __global__ void __launch_bounds__(THREADS, Plan<SPLIT>::MIN_BLOCKS)
             }
             if (i >= 0 && *abort == 0) {
                 if (cprev != 0.f) {  // add the first pass's output with its log-sum-exp weight
-                    if (SPLIT) {
-                        const float4 *src = reinterpret_cast<const float4 *>(p.o_prev_f32 + rowoff * 64 + 32 * h);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.o_prev_f32 + rowoff * 64 + 32 * h);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 q = src[j];
-                            acc[4 * j] += cprev * q.x;
-                            acc[4 * j + 1] += cprev * q.y;
-                            acc[4 * j + 2] += cprev * q.z;
-                            acc[4 * j + 3] += cprev * q.w;
-                        }
-                    } else {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * 64 + 32 * h);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint4 q = src[j];
-                            const uint32_t pw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                acc[8 * j + 2 * e] += cprev * bf16_lo(pw[e]);
-                                acc[8 * j + 2 * e + 1] += cprev * bf16_hi(pw[e]);
-                            }
-                        }
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 q = src[j];
+                        acc[4 * j] += cprev * q.x;
+                        acc[4 * j + 1] += cprev * q.y;
+                        acc[4 * j + 2] += cprev * q.z;
+                        acc[4 * j + 3] += cprev * q.w;
                     }
                 }
                 // one row, this warpgroup's 32 columns, straight to global memory: the first
                 // pass's values of these columns were read above by this same thread
-                if (SPLIT) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.o_f32 + rowoff * 64 + 32 * h);
+                float4 *dst = reinterpret_cast<float4 *>(p.o_f32 + rowoff * 64 + 32 * h);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + rowoff * 64 + 32 * h);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_uint4(pack_bf16(acc[8 * j], acc[8 * j + 1]), pack_bf16(acc[8 * j + 2], acc[8 * j + 3]),
-                                            pack_bf16(acc[8 * j + 4], acc[8 * j + 5]),
-                                            pack_bf16(acc[8 * j + 6], acc[8 * j + 7]));
-                }
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
                 if (h == 0) p.lse[rowoff] = lse2 * LN2;
             }
             T += U.nkt;
@@ -571,21 +548,20 @@ int sm_count()
     return n;
 }
 
-template <bool SPLIT>
-cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t s)
+cudaError_t launch_fwd_split(const FwdParams &p, cudaStream_t s)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Plan<SPLIT>::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(fwd_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Plan::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const int64_t units = static_cast<int64_t>(p.nitems) * p.batch;
     if (units == 0) return cudaSuccess;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * Plan<SPLIT>::MIN_BLOCKS;
+    const int64_t cap = sm_count();
     const unsigned grid = static_cast<unsigned>(units < cap ? units : cap);
-    fwd_kernel<SPLIT><<<grid, THREADS, Plan<SPLIT>::SMEM_BYTES, s>>>(p);
+    fwd_split_kernel<<<grid, THREADS, Plan::SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -593,7 +569,7 @@ cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t s)
 
 cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s)
 {
-    return split ? launch_fwd_t<true>(p, s) : launch_fwd_bf16(p, s);
+    return split ? launch_fwd_split(p, s) : launch_fwd_bf16(p, s);
 }
 
 }  // namespace st
