@@ -55,6 +55,7 @@ def _L():
         common = [p, p, p, i64, i64, i64, i64, p, p, i64, i64]
         lib.oracle_fwd.argtypes = common + [p, p]
         lib.oracle_fwd_rows.argtypes = common + [i64, p, p, p]
+        lib.oracle_decode.argtypes = common + [i64, p, p]
         bcommon = [p, p, p, p, i64, i64, i64, i64, p, p, i64, i64]
         lib.oracle_bwd.argtypes = bcommon + [p, p, p]
         lib.oracle_bwd_rows.argtypes = bcommon + [i64, p, p, p, p]
@@ -132,6 +133,19 @@ class Problem:
         _L().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, _ptr(self.kind),
                              _ptr(self.off), self.l, self.c, len(rows), _ptr(rows), _ptr(o),
                              _ptr(lse))
+        return o, lse
+
+    def decode(self, q, k, v, pos):
+        """One query row per (batch, head) at position pos against the cache rows 0..pos.
+        q: [B, H, d]; k, v: [B, H, n, d].  Returns o [B, H, d], lse [B, H]."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, n, d = k.shape
+        if q.shape != (B, H, d) or not 0 <= pos < n:
+            raise ValueError("q must be [B, H, d] and 0 <= pos < n")
+        o = np.empty_like(q)
+        lse = np.empty((B, H), dtype=np.float64)
+        _L().oracle_decode(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, _ptr(self.kind), _ptr(self.off),
+                           self.l, self.c, int(pos), _ptr(o), _ptr(lse))
         return o, lse
 
     def bwd(self, q, k, v, do):

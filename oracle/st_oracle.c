@@ -117,8 +117,9 @@ int oracle_head_kinds(int family, int head_mode, int num_heads, int64_t l, int64
  * two-pass softmax  m = max_j S_ij, Z = sum_j exp(S_ij - m), P_ij = exp(S_ij - m) / Z, and
  * O_i = sum_j P_ij v_j, lse_i = m + ln Z ([G] §02).  Reading for a row with no allowed key
  * ([G] §02 warns such a row has no softmax): O_i = 0 and lse_i = -inf.
- * qh, kh, vh point at the (batch, head) slab of n x d values.  set and s are scratch of n. */
-static void fwd_row(const double *qh, const double *kh, const double *vh, int64_t n, int64_t d,
+ * qi is the query row; kh, vh point at the (batch, head) slab of n x d values.  set and s are
+ * scratch of n. */
+static void fwd_row(const double *qi, const double *kh, const double *vh, int64_t n, int64_t d,
                     int kind, int64_t l, int64_t c, int64_t o, int64_t i, int64_t *set, double *s,
                     double *orow, double *lse)
 {
@@ -129,7 +130,7 @@ static void fwd_row(const double *qh, const double *kh, const double *vh, int64_
     const double scale = 1.0 / sqrt((double)d);
     double m = -INFINITY;
     for (int64_t a = 0; a < cnt; ++a) {
-        const double *qi = qh + i * d, *kj = kh + set[a] * d;
+        const double *kj = kh + set[a] * d;
         double acc = 0.0;
         for (int64_t t = 0; t < d; ++t) acc += qi[t] * kj[t];
         s[a] = acc * scale;
@@ -157,8 +158,8 @@ void oracle_fwd(const double *q, const double *k, const double *v, int64_t B, in
         for (int64_t r = 0; r < B * H * n; ++r) {
             const int64_t bh = r / n, i = r % n, h = bh % H;
             const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            fwd_row(q + base, k + base, v + base, n, d, kind[h], l, c, off[h], i, set, s,
-                    o + (size_t)r * (size_t)d, lse + r);
+            fwd_row(q + base + (size_t)i * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], i,
+                    set, s, o + (size_t)r * (size_t)d, lse + r);
         }
         free(set);
         free(s);
@@ -180,8 +181,34 @@ void oracle_fwd_rows(const double *q, const double *k, const double *v, int64_t 
         for (int64_t a = 0; a < nrows; ++a) {
             const int64_t r = rows[a], bh = r / n, i = r % n, h = bh % H;
             const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            fwd_row(q + base, k + base, v + base, n, d, kind[h], l, c, off[h], i, set, s,
-                    o_rows + (size_t)a * (size_t)d, lse_rows + a);
+            fwd_row(q + base + (size_t)i * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], i,
+                    set, s, o_rows + (size_t)a * (size_t)d, lse_rows + a);
+        }
+        free(set);
+        free(s);
+    }
+}
+
+/* Decode step: one new query row per (batch, head) at position pos, against the cached keys and
+ * values of rows 0..pos (the sampling setting of [R] §2/§3, where each generated position attends
+ * to its allowed set among the positions already produced).  By the definition of A(pos) (a
+ * subset of {j <= pos}) this is exactly row pos of the forward pass: the same fwd_row, with the
+ * query taken from q[b, h] instead of Q[b, h, pos].  q, o: B x H x d; k, v: B x H x n x d (rows
+ * past pos are never read); lse: B x H. */
+void oracle_decode(const double *q, const double *k, const double *v, int64_t B, int64_t H, int64_t n,
+                   int64_t d, const int *kind, const int64_t *off, int64_t l, int64_t c, int64_t pos,
+                   double *o, double *lse)
+{
+#pragma omp parallel
+    {
+        int64_t *set = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+        double *s = (double *)malloc(sizeof(double) * (size_t)n);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < B * H; ++bh) {
+            const int64_t h = bh % H;
+            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
+            fwd_row(q + (size_t)bh * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], pos, set, s,
+                    o + (size_t)bh * (size_t)d, lse + bh);
         }
         free(set);
         free(s);
