@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode step (one query row per batch-head at the last position) "
+                         "instead of the forward + backward step")
     return ap.parse_args()
 
 
@@ -451,6 +454,69 @@ def run_e2e(args, w, lay, device, stream, flops, world):
             "api": "block_sparse_factorized_b200.st_attn_fwd / st_attn_bwd (C ABI), pinned host buffers"}
 
 
+def run_decode(args, rank, world, local):
+    """The decode step of the workload's pattern at the last position, pos = n - 1 (the largest
+    allowed sets of the growing kinds): one query row per (batch, head) against the K/V caches.
+    HBM-bound, so the metric is the algorithmic bytes per step (the allowed K and V rows, the
+    query and output rows, lse) over its event time, against the measured copy bandwidth."""
+    import ctypes
+
+    import block_sparse_factorized_b200 as bsf
+    w = WORKLOADS[args.workload]
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c)
+    q, k, v, _ = (t.to(device) for t in make_inputs(w))
+    pos = w.n - 1
+    qrow = q[:, :, pos].contiguous()
+    esz = q.element_size()
+    rows = sum(len(lay.decode_row_keys(h, pos)) for h in range(w.heads)) * w.batch
+    nbytes = rows * 2 * 64 * esz + w.batch * w.heads * (2 * 64 * esz + 4)
+    o = torch.empty_like(qrow)
+    lse = torch.empty(qrow.shape[:2], dtype=torch.float32, device=device)
+    ws = torch.empty(max(256, int(lay._lib.st_attn_decode_workspace_bytes(ctypes.byref(bsf._desc(q)), lay.handle))),
+                     dtype=torch.uint8, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        bsf.st_attn_decode(qrow, k, v, lay, pos, o=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_(); flush_rd.sum(); step()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with sampler:
+        for a, b in ev:
+            flush.zero_(); flush_rd.sum()
+            a.record(stream); step(); b.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world, device)
+    peaks = measured_peaks()
+    gbs = nbytes * world / (ms / 1e3) / 1e9
+    line = {"metric": "decode step GB/s (allowed K/V rows + q, o, lse)", "value": gbs, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": f"decode_{w.name}", "pos": pos, "batch": w.batch, "heads": w.heads,
+                       "kv_rows_read": rows, "l2": "flushed before every timed step"},
+            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / world / peaks["hbm_gbs"], "traffic": None},
+            "gpu_launches": 2 * args.steps, "clocks": sampler.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del lay
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -459,6 +525,8 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device; this benchmark times the B200 kernels"}))
         return 1
+    if args.decode:
+        return run_decode(args, rank, world, local)
     return run_ours(args, rank, world, local)
 
 

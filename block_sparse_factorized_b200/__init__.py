@@ -24,7 +24,7 @@ from ._abi import (ST_BF16, ST_FIXED, ST_FP32, ST_KIND_FA1, ST_KIND_FA2, ST_KIND
                    ST_SINGLE_A2, ST_STRIDED, StError)
 
 __all__ = [
-    "Layout", "st_attn_fwd", "st_attn_bwd", "st_attn_fwd_workspace_bytes",
+    "Layout", "st_attn_fwd", "st_attn_bwd", "st_attn_decode", "st_attn_fwd_workspace_bytes",
     "st_attn_bwd_workspace_bytes", "SparseAttention", "StError", "ST_STRIDED", "ST_FIXED",
     "ST_PER_HEAD_ALTERNATING", "ST_MERGED", "ST_SINGLE_A1", "ST_SINGLE_A2", "ST_BF16", "ST_FP32",
     "ST_KIND_SA1", "ST_KIND_SA2", "ST_KIND_SU", "ST_KIND_FA1", "ST_KIND_FA2", "ST_KIND_FU",
@@ -98,6 +98,14 @@ class Layout:
         cnt = _c.c_int64()
         _abi.check(self._lib.st_layout_exec_row(self._h, head, i, keys.ctypes.data_as(_c.c_void_p),
                                                 _c.byref(cnt)), "st_layout_exec_row")
+        return keys[:cnt.value].copy()
+
+    def decode_row_keys(self, head: int, pos: int) -> np.ndarray:
+        """The cache rows the decode step reads for `head` at position `pos` (increasing)."""
+        keys = np.empty(pos + 1, dtype=np.int64)
+        cnt = _c.c_int64()
+        _abi.check(self._lib.st_decode_row_keys(self._h, head, pos, keys.ctypes.data_as(_c.c_void_p),
+                                                _c.byref(cnt)), "st_decode_row_keys")
         return keys[:cnt.value].copy()
 
     def check(self, stream=None) -> None:
@@ -186,6 +194,29 @@ def st_attn_bwd(q, k, v, o, lse, do, layout: Layout, dq=None, dk=None, dv=None, 
                                  workspace.numel(), _c.byref(desc), _stream(stream))
     _abi.check(st, "st_attn_bwd")
     return dq, dk, dv
+
+
+def st_attn_decode(q, k_cache, v_cache, layout: Layout, pos: int, o=None, lse=None, workspace=None,
+                   stream=None):
+    """Decode step: q [B, H, 64] at position pos against k_cache, v_cache [B, H, n, 64] (rows past
+    pos unread).  Returns o [B, H, 64] and lse [B, H] (fp32) -- row pos of the forward pass."""
+    _check_tensors(k_cache, v_cache)
+    if not (q.is_cuda and q.is_contiguous() and q.dtype == k_cache.dtype and q.device == k_cache.device
+            and q.dim() == 3 and tuple(q.shape) == (k_cache.shape[0], k_cache.shape[1], k_cache.shape[3])):
+        raise ValueError("q must be a contiguous [B, H, 64] CUDA tensor matching the caches")
+    desc = _desc(k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    ws = int(layout._lib.st_attn_decode_workspace_bytes(_c.byref(desc), layout.handle))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device)
+    st = layout._lib.st_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), layout.handle, int(pos), _ptr(o),
+                                    _ptr(lse), _ptr(workspace), workspace.numel(), _c.byref(desc),
+                                    _stream(stream))
+    _abi.check(st, "st_attn_decode")
+    return o, lse
 
 
 class SparseAttention(torch.autograd.Function):

@@ -28,6 +28,7 @@ EXPORTED = (
     "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_layout_destroy",
     "st_attn_fwd_workspace_bytes", "st_attn_bwd_workspace_bytes", "st_attn_fwd", "st_attn_bwd",
     "st_attn_bwd_prepare", "st_attn_bwd_main", "st_attn_bwd_finish", "st_attn_bwd_noalloc",
+    "st_attn_decode_workspace_bytes", "st_attn_decode", "st_decode_row_keys",
     "st_status_string", "st_version",
 )
 
@@ -92,12 +93,17 @@ def load() -> ctypes.CDLL:
     lib.st_attn_bwd_finish.argtypes = [P, P, P, sz, pp(st_desc_t), P]
     lib.st_attn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, pp(st_desc_t), P]
     lib.st_attn_bwd_noalloc.restype = i32
+    lib.st_attn_decode_workspace_bytes.argtypes = [pp(st_desc_t), P]
+    lib.st_attn_decode_workspace_bytes.restype = sz
+    lib.st_attn_decode.argtypes = [P, P, P, P, i64, P, P, P, sz, pp(st_desc_t), P]
+    lib.st_decode_row_keys.argtypes = [P, i32, i64, P, pp(i64)]
     lib.st_status_string.argtypes = [i32]
     lib.st_status_string.restype = ctypes.c_char_p
     lib.st_version.restype = ctypes.c_char_p
     for name in ("st_layout_build", "st_layout_upload", "st_layout_head_kind", "st_layout_export",
                  "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_attn_fwd",
-                 "st_attn_bwd", "st_attn_bwd_prepare", "st_attn_bwd_main", "st_attn_bwd_finish"):
+                 "st_attn_bwd", "st_attn_bwd_prepare", "st_attn_bwd_main", "st_attn_bwd_finish",
+                 "st_attn_decode", "st_decode_row_keys"):
         getattr(lib, name).restype = i32
     _lib = lib
     return lib

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include "decode.h"
 #include "kernels.h"
 #include "layout.h"
 
@@ -435,6 +436,65 @@ st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void 
                                stream)) != ST_OK)
         return cs;
     return st_attn_bwd_finish(layout, dq, workspace, workspace_bytes, desc, stream);
+}
+
+size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
+{
+    if (!desc || !layout || desc->batch < 1 || desc->heads < 1 || desc->n < 1) return 0;
+    const size_t nsplit = static_cast<size_t>((desc->n + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
+    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * st::DEC_PART * sizeof(float));
+}
+
+st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache, const st_layout_t *layout,
+                           int64_t pos, void *o, float *lse, void *workspace, size_t workspace_bytes,
+                           const st_desc_t *desc, st_stream_t stream)
+{
+    if (!q || !k_cache || !v_cache || !o || !lse || !layout || !desc) return ST_ERR_INVALID_ARG;
+    const st_layout &L = *layout;
+    if (desc->reserved != 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
+        return ST_ERR_INVALID_ARG;
+    if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
+    if (desc->heads != L.pat.num_heads || desc->n != L.n || pos < 0 || pos >= L.n) return ST_ERR_INVALID_ARG;
+    if (desc->d != 64 || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
+        return ST_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < st_attn_decode_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ST_ERR_ALIGNMENT;
+    st::DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.o = o;
+    p.lse = lse;
+    p.part = static_cast<float *>(workspace);
+    int64_t most = 1;
+    for (int32_t h = 0; h < desc->heads; ++h) {
+        p.kind[h] = L.head_kind[h];
+        p.off[h] = L.head_off[h];
+        const int64_t cnt = st::key_count(st::key_set(p.kind[h], pos, L.l, L.c, p.off[h]));
+        if (cnt > most) most = cnt;
+    }
+    p.pos = pos;
+    p.n = L.n;
+    p.l = L.l;
+    p.c = L.c;
+    p.bh = static_cast<int32_t>(desc->batch * desc->heads);
+    p.heads = static_cast<int32_t>(desc->heads);
+    p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
+    const int32_t nsplit = static_cast<int32_t>((most + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
+    return st::launch_decode(p, nsplit, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+}
+
+st_status_t st_decode_row_keys(const st_layout_t *layout, int32_t head, int64_t pos, int64_t *keys, int64_t *count)
+{
+    if (!layout || !keys || !count || head < 0 || head >= layout->pat.num_heads || pos < 0 || pos >= layout->n)
+        return ST_ERR_INVALID_ARG;
+    const st::KeySet ks = st::key_set(layout->head_kind[head], pos, layout->l, layout->c, layout->head_off[head]);
+    const int64_t cnt = st::key_count(ks);
+    for (int64_t e = 0; e < cnt; ++e) keys[e] = st::key_at(ks, e);
+    *count = cnt;
+    return ST_OK;
 }
 
 const char *st_status_string(st_status_t s)

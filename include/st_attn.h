@@ -232,6 +232,36 @@ ST_API st_status_t st_attn_bwd_noalloc(const void *q, const void *k, const void 
                                        const st_layout_t *layout, void *dq, void *dk, void *dv,
                                        const st_desc_t *desc, st_stream_t stream);
 
+/* Decode step ("长序列为何不必让每个 token 看见全部历史？…" §11: incremental inference brings one new
+ * query row per step, Q_LEN = 1, against the key/value cache including the new position).
+ * For every (batch, head): the query row q[b, h] at sequence position pos attends to its allowed
+ * set A(h, pos) among the cache rows 0..pos -- by the set definitions exactly row pos of
+ * st_attn_fwd on the full sequence.  Scores and the softmax are computed in fp32 ("Sparse
+ * Transformers 深度解读报告" §3.6: query-key products in fp32 when sampling).
+ *   q:        [batch, heads, 64] (desc->dtype)
+ *   k_cache,
+ *   v_cache:  [batch, heads, n, 64], n = the layout's n (the cache capacity); rows past pos are
+ *             not read
+ *   o:        [batch, heads, 64] output (desc->dtype);  lse: [batch, heads] fp32 output (natural
+ *             log; -inf for a row with no allowed key, whose o is 0)
+ *   workspace: st_attn_decode_workspace_bytes (per-chunk partial results), 256-byte aligned
+ * desc is the full-sequence descriptor (its n is the cache capacity).  The layout need not be
+ * uploaded: the kernels read only the per-head set kinds, passed by value.  Errors:
+ * ST_ERR_INVALID_ARG (NULL pointers, pos outside [0, n), heads or n not the layout's),
+ * ST_ERR_UNSUPPORTED (d != 64, more than 64 heads), ST_ERR_ALIGNMENT, ST_ERR_WORKSPACE,
+ * ST_ERR_CUDA. */
+ST_API size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout);
+ST_API st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                                  const st_layout_t *layout, int64_t pos, void *o, float *lse,
+                                  void *workspace, size_t workspace_bytes, const st_desc_t *desc,
+                                  st_stream_t stream);
+
+/* Host enumeration of the cache rows the decode step reads for head `head` at position pos,
+ * increasing, written to keys[0 .. *count-1]; keys must hold pos + 1 entries.  For tests of the
+ * decode step's key sets against the set definitions. */
+ST_API st_status_t st_decode_row_keys(const st_layout_t *layout, int32_t head, int64_t pos,
+                                      int64_t *keys, int64_t *count);
+
 /* Static description of a status code. */
 ST_API const char *st_status_string(st_status_t status);
 

@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 
 import oracle
-from workloads import ALTERNATING, FIXED, MERGED, WORKLOADS
+from workloads import ALTERNATING, FIXED, MERGED, STRIDED, WORKLOADS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -235,3 +235,19 @@ def test_dq_direct_heads():
     assert bsf.Layout(FIXED, ALTERNATING, 2, 1024, 256, 32).info()["dq_direct_heads"] == 0
     # merged fixed heads: same-block pass plus the earlier blocks' summaries (two items per tile)
     assert bsf.Layout(FIXED, MERGED, 2, 1024, 128, 32).info()["dq_direct_heads"] == 0
+
+
+@pytest.mark.parametrize("family,mode,H,n,l,c", [
+    (STRIDED, ALTERNATING, 2, 512, 16, 0), (STRIDED, MERGED, 2, 512, 16, 0), (STRIDED, MERGED, 1, 384, 128, 0),
+    (FIXED, ALTERNATING, 6, 512, 16, 4), (FIXED, MERGED, 4, 512, 16, 4), (FIXED, ALTERNATING, 4, 1024, 128, 32),
+    (FIXED, MERGED, 2, 1024, 128, 32)])
+def test_decode_row_keys_match_sets(family, mode, H, n, l, c):
+    """The cache rows the decode step reads are exactly the oracle's A(h, pos), in order."""
+    lay = bsf.Layout(family, mode, H, n, l, c)
+    rows = sorted(set(list(range(0, 2 * l + 3)) + np.linspace(0, n - 1, 40).astype(int).tolist()))
+    for h in range(H):
+        kind, o = lay.head_kind(h)
+        for pos in rows:
+            got = lay.decode_row_keys(h, pos)
+            want = oracle.row_set(kind, pos, l, c, o)
+            assert np.array_equal(got, want), (h, kind, o, pos)
