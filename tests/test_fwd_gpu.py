@@ -34,8 +34,10 @@ SMALL = [
     Workload("f_n1024_l256_c8", FIXED, ALTERNATING, 1024, 256, 8, 1, 4),
     Workload("f_single_a2_n512_l32_c4", FIXED, SINGLE_A2, 512, 32, 4, 1, 8),
     Workload("f_merged_n1024_l128_c32", FIXED, MERGED, 1024, 128, 32, 1, 4),
-    # long backward items: summary key tile 0 is read by all 64 query tiles
-    Workload("f_n8192_l128_c32_long", FIXED, ALTERNATING, 8192, 128, 32, 1, 2),
+    # long backward items: summary key tile 0 is read by 96 query tiles, more than one backward
+    # chunk (64), so its dK/dV are the sum of two chunks' partials -- also in a merge pass
+    Workload("f_n12288_l128_c32_long", FIXED, ALTERNATING, 12288, 128, 32, 1, 2),
+    Workload("f_merged_n12288_l128_c32_long", FIXED, MERGED, 12288, 128, 32, 1, 1),
     # degenerate sets: c = l (pattern 2 reads every earlier key), c = 128 with three head-2
     # offsets, fixed head 1 alone, odd batch and head counts
     Workload("f_n512_l128_c128", FIXED, ALTERNATING, 512, 128, 128, 1, 2),
@@ -74,7 +76,7 @@ FP32 = [WORKLOADS["strided_n256_l16_fp32"],
         Workload("f32_fixed_n512_l128_c32", FIXED, ALTERNATING, 512, 128, 32, 1, 4, dtype="fp32"),
         Workload("f32_s_merged_n768_l24", STRIDED, MERGED, 768, 24, 0, 1, 2, dtype="fp32"),
         Workload("f32_f_merged_n512_l128_c32", FIXED, MERGED, 512, 128, 32, 1, 2, dtype="fp32"),
-        Workload("f32_fixed_n8192_l128_c32_long", FIXED, SINGLE_A2, 8192, 128, 32, 1, 1, dtype="fp32")]
+        Workload("f32_fixed_n12288_l128_c32_long", FIXED, SINGLE_A2, 12288, 128, 32, 1, 1, dtype="fp32")]
 
 
 @pytest.mark.parametrize("w", FP32, ids=lambda w: w.name)
