@@ -410,8 +410,10 @@ st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *worksp
     cv.dq_acc = ws.dq_acc;
     cv.dq = static_cast<uint16_t *>(dq);
     cv.dq_f32 = static_cast<float *>(dq);
-    cv.head_flags = layout->d_head_flags;
-    cv.bh = desc->batch * desc->heads;
+    cv.nacc = 0;
+    for (int32_t h = 0; h < desc->heads; ++h)
+        if (!(layout->head_flags[h] & st::HEAD_DQ_DIRECT)) cv.acc_head[cv.nacc++] = h;
+    cv.batch = static_cast<int32_t>(desc->batch);
     cv.n = static_cast<int32_t>(desc->n);
     cv.heads = static_cast<int32_t>(desc->heads);
     return st::launch_dq_convert(cv, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;

@@ -105,14 +105,17 @@ __global__ void __launch_bounds__(256, 4) bwd_pre_kernel(const PreParams p)
     }
 }
 
-// Same grid as bwd_pre_kernel; a thread converts UNROLL groups of 8 consecutive values, 256
-// groups apart.
+// Grid: x over chunks of one batch-head, y over (batch, accumulated head) pairs only -- the
+// heads whose dQ the main kernel stores directly get no block.  A thread converts UNROLL groups of
+// 8 consecutive values, 256 groups apart.
 template <bool F32>
 __global__ void __launch_bounds__(256, 4) dq_convert_kernel(const ConvParams p)
 {
     const int64_t n8 = static_cast<int64_t>(p.n) * 8;  // 8-value groups per batch-head
-    for (int64_t bh = blockIdx.y; bh < p.bh; bh += gridDim.y) {
-        if (p.head_flags[bh % p.heads] & HEAD_DQ_DIRECT) continue;  // written by the main kernel
+    const int64_t pairs = static_cast<int64_t>(p.batch) * p.nacc;
+    for (int64_t y = blockIdx.y; y < pairs; y += gridDim.y) {
+        const int64_t b = y / p.nacc;
+        const int64_t bh = b * p.heads + p.acc_head[y - b * p.nacc];
         const float4 *src = reinterpret_cast<const float4 *>(p.dq_acc) + bh * n8 * 2;
         for (int64_t a0 = static_cast<int64_t>(blockIdx.x) * blockDim.x * UNROLL + threadIdx.x; a0 < n8;
              a0 += static_cast<int64_t>(gridDim.x) * blockDim.x * UNROLL) {
@@ -280,7 +283,9 @@ cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s)
 
 cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s)
 {
-    const dim3 grid = head_grid((static_cast<int64_t>(p.n) * 8 + 256 * UNROLL - 1) / (256 * UNROLL), p.bh);
+    if (p.nacc == 0) return cudaSuccess;
+    const dim3 grid = head_grid((static_cast<int64_t>(p.n) * 8 + 256 * UNROLL - 1) / (256 * UNROLL),
+                                static_cast<int64_t>(p.batch) * p.nacc);
     if (f32)
         dq_convert_kernel<true><<<grid, 256, 0, s>>>(p);
     else

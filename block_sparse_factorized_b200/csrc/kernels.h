@@ -75,9 +75,9 @@ struct ConvParams {
     const float *dq_acc;
     uint16_t *dq;
     float *dq_f32;               // fp32 I/O: plain copy instead of rounding to bf16
-    const int32_t *head_flags;   // [H]: heads with HEAD_DQ_DIRECT are skipped
-    int64_t bh;                  // B*H
-    int32_t n, heads;
+    int32_t acc_head[64];        // the heads whose dQ is accumulated (not HEAD_DQ_DIRECT)
+    int32_t nacc;                // how many
+    int32_t batch, n, heads;
 };
 
 // dK/dV of split key tiles: sum of the chunks' fp32 partials in chunk order, plus the first
