@@ -108,6 +108,38 @@ bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_
     return true;
 }
 
+// bf16 [BH, n, 64] maps with 16-column (32-byte, 32-byte swizzle), 32-row boxes in the natural,
+// grid-column and summary frames: one backward warp's slice of a dK or dV tile.
+bool make_maps_warp16(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum)
+{
+    memset(&m, 0, sizeof(m));
+    const cuuint64_t row = 64 * 2, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
+    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    {
+        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[2] = {row, n * row};
+        const cuuint32_t box[3] = {16, 32, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+    }
+    if (col) {
+        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[3] = {l * row, row, n * row};
+        const cuuint32_t rows = static_cast<cuuint32_t>(g.Rt < 32 ? g.Rt : 32);
+        const cuuint32_t slots = static_cast<cuuint32_t>(g.Rt < 32 ? 32 / g.Rt : 1);
+        const cuuint32_t box[4] = {16, rows, slots, 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+    }
+    if (sum) {
+        const cuuint64_t dims[4] = {64, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
+        const cuuint64_t str[3] = {row, l * row, n * row};
+        const cuuint32_t rows = static_cast<cuuint32_t>(g.c < 32 ? g.c : 32);
+        const cuuint32_t runs = static_cast<cuuint32_t>(g.c < 32 ? 32 / g.c : 1);
+        const cuuint32_t box[4] = {16, rows, runs, 1};
+        if (!encode(&m.sum, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+    }
+    return true;
+}
+
 // The dQ output in the natural frame with a 16-column, 32-row box: one warp's slice of a query
 // tile whose dQ the backward kernel stores directly (fp32: 64-byte swizzle, as the accumulator's
 // reduce map; bf16: 32-byte rows, 32-byte swizzle).
@@ -351,7 +383,8 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
     }
     if (!make_map_dq_direct(&p.dq_direct, dq, L.geom, BH, f32)) return ST_ERR_CUDA;
     if (!make_maps_f32(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol)) return ST_ERR_CUDA;
-    if (!f32 && (!make_maps(p.dk, dk, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.dv, dv, L.geom, BH, f.kcol, f.ksum)))
+    if (!f32 && (!make_maps_warp16(p.dk_w, dk, L.geom, BH, f.kcol, f.ksum) ||
+                 !make_maps_warp16(p.dv_w, dv, L.geom, BH, f.kcol, f.ksum)))
         return ST_ERR_CUDA;
     if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false) ||
         !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum))

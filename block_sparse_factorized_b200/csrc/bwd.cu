@@ -12,8 +12,10 @@
 // with TMA reduce-adds.
 //
 // The kernel is persistent (one CTA per SM) and claims items, longest first, from a global
-// counter.  K and V have two buffers, so the next item's loads and first S, dP products overlap
-// the current item's last tiles and its dK/dV epilogue.  Roles (608 threads):
+// counter.  Both the MMA issuer and the softmax warps walk one flat sequence of query tiles over
+// all the items they claim, so the next item's S and dP (K and V have two buffers) and its first P
+// overlap the current item's last tile and its dK/dV epilogue, even for an item of one tile.
+// Roles (576 threads):
 //   warp 0      TMA: K and V of each item (KVS slots), Q and dO per query tile (2-stage ring)
 //   warp 1      MMA issuer: S = Q K^T and dP = dO V^T (TMEM, 128 x 128 fp32 each), then after
 //               the softmax warps wrote P and dS (bf16, SMEM): dV += P^T dO, dK += dS^T Q
@@ -22,11 +24,10 @@
 //               32g..32g+31 (no row reduction is needed here: P comes from the saved lse):
 //               interval mask, P, dS; dQ columns 16g.. staged per warp and added to the fp32
 //               accumulator with a TMA reduce (or, where this item is the only one that reads
-//               the query tile, written to dQ directly); at the end of an item one key row per thread:
-//               dK, dV columns 16g.. staged in SMEM for a TMA store (bf16), written row by row
-//               (fp32), or stored as the fp32 partial of a split key tile.
-//   warp 18     (bf16) the TMA stores of the staged dK, dV tiles, so that no softmax warp waits
-//               for them.
+//               the query tile, written to dQ directly); at the end of an item one key row per
+//               thread: dK, dV columns 16g.. staged per warp (32 rows) in the warp's dQ slot for
+//               two TMA stores (bf16), written row by row (fp32), or stored as the fp32 partial
+//               of a split key tile.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
 #include "tiles.cuh"
 
@@ -49,8 +50,7 @@ constexpr uint32_t OFF_ITEMS = OFF_BAR + 256;      // the claimed items' fields,
 constexpr uint32_t SMEM_BYTES = OFF_ITEMS + NSCHED * 96;
 constexpr int NWG = 4;                             // softmax warpgroups
 constexpr int NSM = 128 * NWG;                     // softmax threads
-constexpr int STORE_WARP = 2 + NSM / 32;           // the last warp
-constexpr int THREADS = 64 + NSM + 32;
+constexpr int THREADS = 64 + NSM;
 constexpr int CW = 128 / NWG;                      // score columns per warpgroup (32)
 constexpr int OW = 64 / NWG;                       // dQ / dK / dV columns per warpgroup (16)
 constexpr uint32_t TMEM_COLS = 512;
@@ -62,10 +62,8 @@ struct Bars {
     uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
     uint64_t acc_free;             // the epilogue has read dK and dV of the item from TMEM
     uint64_t mma_idle;             // every MMA this CTA issued has completed (before teardown)
-    uint64_t stage_full, stage_free;  // bf16 dK/dV staged in the P area / its TMA store has read it
     uint64_t sched_full[NSCHED], sched_empty[NSCHED];
     int32_t sched[NSCHED];         // claimed item (index into items x batch), -1 = none left
-    int32_t store[4];              // staged tile: key frame, offset, key tile, batch-head (-1: end)
     uint32_t tmem_base;
     int32_t abort;
 };
@@ -135,8 +133,6 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, NSM);
         mbar_init(&bars->acc_free, NSM);
-        mbar_init(&bars->stage_full, NSM);
-        mbar_init(&bars->stage_free, 1);
         mbar_init(&bars->mma_idle, 1);
         for (int s = 0; s < NSCHED; ++s) {
             mbar_init(&bars->sched_full[s], 1);
@@ -237,29 +233,38 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                                 desc_sw128(v + 32 * kk, 16, 1024), id_nn, kk > 0 ? 1u : 0u);
                 mma_commit(&bars->dp_full);
             };
-            int32_t I = 0, J = 0;
-            bool fail = false;
-            for (int32_t j = 0; !fail; ++j) {
-                const int32_t u = next_item(bars, j, false, abort, p.err);
-                if (u < 0) break;
-                const int32_t nq = (reinterpret_cast<const Item *>(smem + OFF_ITEMS) + j % NSCHED)->nq;
-                const int ks = I % KVS;
-                const uint32_t sK = smem_u32(smem + OFF_K + ks * TB), sV = smem_u32(smem + OFF_V + ks * TB);
-                if (!mbar_wait(&bars->kv_full[ks], (I / KVS) & 1, abort, p.err) ||
-                    !mbar_wait(&bars->qdo_full[J % NST], (J / NST) & 1, abort, p.err))
-                    break;
-                tc_fence_after();
-                issue_s(sQ(J), sK);
-                issue_dp(sDO(J), sV);
-                for (int32_t jj = 0; jj < nq; ++jj) {
-                    const int32_t t = J + jj;
-                    const bool next = jj + 1 < nq;
-                    if (!mbar_wait(&bars->p_ready, t & 1, abort, p.err)) { fail = true; break; }
-                    // the previous item's epilogue must have read dK and dV before they restart
-                    if (jj == 0 && I > 0 && !mbar_wait(&bars->acc_free, (I - 1) & 1, abort, p.err)) {
-                        fail = true;
-                        break;
+            // One flat loop over the query tiles of all items this CTA claims: the tile after the
+            // last one of an item is the next item's first, so the next item's S and dP are
+            // issued as early as within an item (after dV and after dK, dQ of the current tile).
+            auto item_nq = [&](int32_t jj_slot) {
+                return (reinterpret_cast<const Item *>(smem + OFF_ITEMS) + jj_slot % NSCHED)->nq;
+            };
+            int32_t j = 0, I = 0, J = 0;  // current item (claim index), items started, tiles done
+            int32_t u = next_item(bars, 0, false, abort, p.err);
+            if (u >= 0) {
+                int32_t nq = item_nq(0), jj = 0, ks = 0;
+                bool ok = mbar_wait(&bars->kv_full[0], 0, abort, p.err) &&
+                          mbar_wait(&bars->qdo_full[0], 0, abort, p.err);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(sQ(0), smem_u32(smem + OFF_K));
+                    issue_dp(sDO(0), smem_u32(smem + OFF_V));
+                }
+                while (ok) {
+                    const int32_t t = J;
+                    const bool last = jj + 1 == nq;
+                    // the next tile: this item's next query tile, or the next item's first
+                    int32_t nks = ks;
+                    bool has_next = !last;
+                    if (last) {
+                        const int32_t un = next_item(bars, j + 1, false, abort, p.err);
+                        if (un == -2) break;
+                        has_next = un >= 0;
+                        nks = (I + 1) % KVS;
                     }
+                    if (!mbar_wait(&bars->p_ready, t & 1, abort, p.err)) break;
+                    // the previous item's epilogue must have read dK and dV before they restart
+                    if (jj == 0 && I > 0 && !mbar_wait(&bars->acc_free, (I - 1) & 1, abort, p.err)) break;
                     tc_fence_after();
                     // dV += P^T dO: A = P^T MN-major (two 64-key atoms 16 KB apart), B = dO
                     // MN-major; 16 queries (2048 bytes) per step
@@ -267,20 +272,18 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + kk * 2048, TB, 1024),
                                     desc_sw128(sDO(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
-                    if (next) {  // S of the next query tile: the softmax warps are done reading S_t
-                        if (!mbar_wait(&bars->qdo_full[(t + 1) % NST], ((t + 1) / NST) & 1, abort, p.err)) {
-                            fail = true;
+                    if (has_next) {  // S of the next tile: the softmax warps are done reading S_t
+                        if (!mbar_wait(&bars->qdo_full[(t + 1) % NST], ((t + 1) / NST) & 1, abort, p.err) ||
+                            (last && !mbar_wait(&bars->kv_full[nks], ((I + 1) / KVS) & 1, abort, p.err)))
                             break;
-                        }
                         tc_fence_after();
-                        issue_s(sQ(t + 1), sK);
+                        issue_s(sQ(t + 1), smem_u32(smem + OFF_K + nks * TB));
                     }
                     if (!mbar_wait(&bars->ds_ready, t & 1, abort, p.err) ||
-                        (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort, p.err))) {
-                        fail = true;
+                        (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort, p.err)))
                         break;
-                    }
                     tc_fence_after();
+                    const uint32_t sK = smem_u32(smem + OFF_K + ks * TB);
                     // dK += dS^T Q (as dV), dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
@@ -290,38 +293,30 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (kk >> 2) * TB + (kk & 3) * 32, 16, 1024),
                                     desc_sw128(sK + kk * 2048, TB, 1024), id_kt, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->dq_full);   // also: dK, dV of the item complete on the last tile
+                    mma_commit(&bars->dq_full);   // also: dK, dV of the item complete on its last tile
                     mma_commit(&bars->qdo_empty[t % NST]);
-                    if (next) issue_dp(sDO(t + 1), sV);  // dP_t already consumed
+                    if (last) {
+                        mma_commit(&bars->kv_empty[ks]);  // K and V of this item are no longer read
+                        done_item(bars, j, false);
+                    }
+                    if (has_next) issue_dp(sDO(t + 1), smem_u32(smem + OFF_V + nks * TB));  // dP_t consumed
+                    ++J;
+                    if (!has_next) break;
+                    if (last) {
+                        ++j;
+                        ++I;
+                        nq = item_nq(j);
+                        jj = 0;
+                        ks = nks;
+                    } else {
+                        ++jj;
+                    }
                 }
-                if (fail) break;
-                mma_commit(&bars->kv_empty[ks]);  // K and V of this item are no longer read
-                done_item(bars, j, false);
-                J += nq;
-                ++I;
             }
             // no product may still be running when TMEM is released (also after an abort)
             mma_commit(&bars->mma_idle);
             volatile int32_t never = 0;
             mbar_wait(&bars->mma_idle, 0, &never, p.err);
-        }
-    } else if (warp == STORE_WARP) {
-        // ---------------- dK, dV tile stores (bf16) ----------------
-        if (!F32 && lane == 0 && run) {
-            // the softmax warps stage one item's tiles at a time; the record says where they go
-            for (int32_t sf = 0;; ++sf) {
-                if (!mbar_wait(&bars->stage_full, sf & 1, abort, p.err)) break;
-                const volatile int32_t *r = bars->store;
-                const int32_t fr = r[0], o = r[1], tile = r[2], bh = r[3];
-                if (tile < 0) break;
-                if (*abort == 0) {
-                    store_tile(p.dk, fr, p.g, o, tile, bh, smem + OFF_P);
-                    store_tile(p.dv, fr, p.g, o, tile, bh, smem + OFF_P + TB);
-                    bulk_commit();
-                    bulk_wait_read_all();  // the next item's P stores may overwrite the staging
-                }
-                mbar_arrive(&bars->stage_free);
-            }
         }
     } else {
         // ------- P, dS, dQ drain, epilogue (warps 2..: warpgroup g owns score columns CW g..) -------
@@ -346,8 +341,6 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         const Item *cur = nullptr;     // the item being processed (its shared slot: the fields
                                        // are read where needed, to keep registers free)
         size_t head_base = 0;          // first row of its batch-head
-        int32_t SF = 0;                // dK/dV tiles staged for a TMA store so far
-        bool stage_pending = false;    // the last item's staging (P area) may still be being read
         // Order per query tile: P_0; then for each t: dS_t, P_{t+1}, drain dQ_t.  Building P_{t+1}
         // while the tensor core computes dK_t and dQ_t hides their latency.  Buffer safety comes
         // from commit order: S_{t+1} is issued after dV_t (so s_full(t+1) means P_t was read) and
@@ -360,19 +353,20 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         // Row data of query tile jj of the item (interval, -lse, -D).  The loads are issued just
         // before the wait for S: issued any earlier they would sit in front of the proxy fences of
         // the dS phase, which wait for them.
-        auto p_phase = [&](int32_t t, int32_t jj) {  // P_t = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
+        auto p_phase = [&](int32_t t, const Item *it, int32_t jj) {  // P_t = exp2(S log2e / sqrt(d) - lse log2e) -> SMEM
             int32_t lo_abs, hi_abs;
-            const int32_t i = row_interval(p.g, cur->part, cur->w.begin + jj, row, lo_abs, hi_abs);
+            const int32_t i = row_interval(p.g, it->part, it->w.begin + jj, row, lo_abs, hi_abs);
+            const size_t hb = static_cast<size_t>(it->bh) * p.g.n;
             nlse = 0.f;
             nD = 0.f;
             if (i >= 0) {
-                const float lse = p.lse[head_base + i];
+                const float lse = p.lse[hb + i];
                 // a row with no allowed key (lse = -inf) has every entry masked to -inf below;
                 // keep its base finite so that -inf + base stays -inf instead of NaN
                 nlse = lse == -INFINITY ? 0.f : -lse * LOG2E;
-                nD = -p.delta[head_base + i] * dsc;
+                nD = -p.delta[hb + i] * dsc;
             }
-            const int32_t base = cur->w.tile * TILE + CW * g;
+            const int32_t base = it->w.tile * TILE + CW * g;
             lo = lo_abs - base;
             hi = hi_abs - base;
             if (!wait_all(&bars->s_full, t & 1)) return;
@@ -392,10 +386,6 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     pr[e] = ex2(x0);
                     pr[e + 1] = ex2(x1);
                 }
-            }
-            if (stage_pending) {  // the previous item's dK/dV staging (P area) has been read
-                stage_pending = false;
-                if (!wait_all(&bars->stage_free, (SF - 1) & 1)) return;
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -465,98 +455,73 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 bulk_commit();
             }
         };
-        int32_t J = 0;  // query tiles processed
-        for (int32_t j = 0; ok; ++j) {
-            const int32_t u = next_item(bars, j, true, abort, p.err);
-            if (u < 0) break;
-            cur = reinterpret_cast<const Item *>(smem + OFF_ITEMS) + j % NSCHED;
+        // One flat loop over the query tiles of all items, as the MMA issuer's: per tile t, dS_t,
+        // then P of the next tile (the next item's first after an item's last tile), then the
+        // drain of dQ_t, and after an item's last tile its dK/dV epilogue -- so that building the
+        // next P covers the wait for dK_t, dQ_t even when an item has a single query tile.
+        int32_t J = 0, j = 0;  // query tiles processed, current item (claim index)
+        const Item *slot0 = reinterpret_cast<const Item *>(smem + OFF_ITEMS);
+        if (next_item(bars, 0, true, abort, p.err) >= 0) {
+            cur = slot0;
             head_base = static_cast<size_t>(cur->bh) * p.g.n;
-            const int32_t nq = cur->nq;
-            p_phase(J, 0);
-            for (int32_t jj = 0; ok && jj < nq; ++jj) {
-                const int32_t t = J + jj;
-                ds_phase(t);
-                if (ok && jj + 1 < nq) p_phase(t + 1, jj + 1);
-                if (ok) drain(t, jj);
-            }
-            if (!ok) break;
-            // ------- dK, dV of the item: one key row per thread, warpgroup g owns columns OW g.. -------
-            // (the last drain waited for dq_full of the item's last tile, whose commit covers
-            // every dK and dV product of the item).  dK and dV are handled one at a time: the next
-            // item's first dV product waits for its P_0, which these threads build afterwards
-            // anyway, so releasing TMEM early would gain nothing.
-            const int32_t pos = frame_pos(p.g, cur->part.kframe, cur->part.o, cur->w.tile, row);
-            // output of one row slice: add the first pass's values for a merge part (read by this
-            // same thread), round, store
-            auto emit = [&](int which, float (&a)[OW]) {
-                const size_t off = (head_base + pos) * 64 + OW * g;
-                if (F32) {
-                    float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + off;
-                    if (cur->part.merge) {
-                        const float4 *src = reinterpret_cast<const float4 *>(of);
-#pragma unroll
-                        for (int q = 0; q < OW / 4; ++q) {
-                            const float4 x = src[q];
-                            a[4 * q] += x.x;
-                            a[4 * q + 1] += x.y;
-                            a[4 * q + 2] += x.z;
-                            a[4 * q + 3] += x.w;
-                        }
+            int32_t nq = cur->nq, jj = 0;
+            p_phase(0, cur, 0);
+            while (ok) {
+                const int32_t t = J;
+                const bool last = jj + 1 == nq;
+                const Item *nxt = cur;
+                int32_t njj = jj + 1;
+                bool has_next = !last;
+                if (last) {
+                    const int32_t un = next_item(bars, j + 1, true, abort, p.err);
+                    if (un == -2) {
+                        ok = false;
+                        break;
                     }
-                    float4 *d4 = reinterpret_cast<float4 *>(of);
+                    has_next = un >= 0;
+                    nxt = slot0 + (j + 1) % NSCHED;
+                    njj = 0;
+                }
+                ds_phase(t);
+                if (ok && has_next) p_phase(t + 1, nxt, njj);
+                if (ok) drain(t, jj);
+                if (!ok) break;
+                if (!last) {
+                    ++J;
+                    ++jj;
+                    continue;
+                }
+                // ------- dK, dV of the item: one key row per thread, warpgroup g owns columns OW g.. -------
+                // (the last drain waited for dq_full of the item's last tile, whose commit covers
+                // every dK and dV product of the item).  The next item's P_0 is already built; its
+                // first dV product waits for acc_free, arrived below.
+                const int32_t pos = frame_pos(p.g, cur->part.kframe, cur->part.o, cur->w.tile, row);
+                // output of one row slice: add the first pass's values for a merge part (read by this
+                // same thread), round, store
+                auto emit = [&](int which, float (&a)[OW]) {
+                    const size_t off = (head_base + pos) * 64 + OW * g;
+                    if (F32) {
+                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + off;
+                        if (cur->part.merge) {
+                            const float4 *src = reinterpret_cast<const float4 *>(of);
 #pragma unroll
-                    for (int q = 0; q < OW / 4; ++q) d4[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-                } else {
-                    uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk_out : p.dv_out) + off);
-                    if (cur->part.merge) {
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const uint4 x = d4[q];
-                            const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                a[8 * q + 2 * e] += bf16_lo(xx[e]);
-                                a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
+                            for (int q = 0; q < OW / 4; ++q) {
+                                const float4 x = src[q];
+                                a[4 * q] += x.x;
+                                a[4 * q + 1] += x.y;
+                                a[4 * q + 2] += x.z;
+                                a[4 * q + 3] += x.w;
                             }
                         }
-                    }
+                        float4 *d4 = reinterpret_cast<float4 *>(of);
 #pragma unroll
-                    for (int q = 0; q < 2; ++q)
-                        d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
-                                           pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
-                }
-            };
-            // Chunk of a split key tile: store the fp32 partial in this chunk's slot (a pass after
-            // the kernel adds the chunks' slots in chunk order and writes dK and dV), in thread
-            // order: uint4 ((which * 4 + q) * 4 + g) * 128 + row, so that each warp store is 512
-            // contiguous bytes.  bf16 output goes through the P area and one TMA store per tile.
-            constexpr size_t SLOT = 2 * 128 * 64;
-            const bool split = cur->w.slot >= 0;
-            const bool staged = !F32 && !split;
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                uint32_t a16[OW];
-                tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
-                tmem_wait_ld();
-                if (*abort != 0) continue;
-                if (split) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.partials + (static_cast<size_t>(cur->w.slot) * p.batch + cur->b) * SLOT);
-#pragma unroll
-                    for (int q = 0; q < OW / 4; ++q)
-                        dst[((which * 4 + q) * 4 + g) * 128 + row] = make_uint4(a16[4 * q], a16[4 * q + 1], a16[4 * q + 2], a16[4 * q + 3]);
-                } else {
-                    float a[OW];
-#pragma unroll
-                    for (int e = 0; e < OW; ++e) a[e] = __uint_as_float(a16[e]);
-                    if (F32) {
-                        if (pos >= 0) emit(which, a);
+                        for (int q = 0; q < OW / 4; ++q) d4[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
                     } else {
-                        if (cur->part.merge && pos >= 0) {  // add the first pass's values
-                            const uint4 *src = reinterpret_cast<const uint4 *>((which == 0 ? p.dk_out : p.dv_out) +
-                                                                               (head_base + pos) * 64 + OW * g);
+                        uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk_out : p.dv_out) + off);
+                        if (cur->part.merge) {
 #pragma unroll
                             for (int q = 0; q < 2; ++q) {
-                                const uint4 x = src[q];
+                                const uint4 x = d4[q];
                                 const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
@@ -565,38 +530,91 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                                 }
                             }
                         }
-                        const uint32_t dst = smem_u32(smem + OFF_P) + which * TB;  // staging: dK, dV tiles
 #pragma unroll
                         for (int q = 0; q < 2; ++q)
-                            st_shared_v4(dst + sw128_off(row, 2 * g + q), pack_bf16(a[8 * q], a[8 * q + 1]),
-                                         pack_bf16(a[8 * q + 2], a[8 * q + 3]), pack_bf16(a[8 * q + 4], a[8 * q + 5]),
-                                         pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+                            d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
+                                               pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+                    }
+                };
+                // Chunk of a split key tile: store the fp32 partial in this chunk's slot (a pass after
+                // the kernel adds the chunks' slots in chunk order and writes dK and dV), in thread
+                // order: uint4 ((which * 4 + q) * 4 + g) * 128 + row, so that each warp store is 512
+                // contiguous bytes.  bf16 output: each warp stages its 32 rows x 16 columns of dK and
+                // dV in its own dQ staging slot and writes them with two TMA stores (no cross-warp
+                // barrier; the warp's next dQ drain waits for their reads as for a reduce).
+                constexpr size_t SLOT = 2 * 128 * 64;
+                const bool split = cur->w.slot >= 0;
+                const bool staged = !F32 && !split;
+                if (staged) {
+                    if (lane == 0) bulk_wait_read_all();  // this warp's last reduce has read the slot
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int which = 0; which < 2; ++which) {
+                    uint32_t a16[OW];
+                    tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
+                    tmem_wait_ld();
+                    if (*abort != 0) continue;
+                    if (split) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.partials + (static_cast<size_t>(cur->w.slot) * p.batch + cur->b) * SLOT);
+#pragma unroll
+                        for (int q = 0; q < OW / 4; ++q)
+                            dst[((which * 4 + q) * 4 + g) * 128 + row] = make_uint4(a16[4 * q], a16[4 * q + 1], a16[4 * q + 2], a16[4 * q + 3]);
+                    } else {
+                        float a[OW];
+#pragma unroll
+                        for (int e = 0; e < OW; ++e) a[e] = __uint_as_float(a16[e]);
+                        if (F32) {
+                            if (pos >= 0) emit(which, a);
+                        } else {
+                            if (cur->part.merge && pos >= 0) {  // add the first pass's values
+                                const uint4 *src = reinterpret_cast<const uint4 *>((which == 0 ? p.dk_out : p.dv_out) +
+                                                                                   (head_base + pos) * 64 + OW * g);
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const uint4 x = src[q];
+                                    const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        a[8 * q + 2 * e] += bf16_lo(xx[e]);
+                                        a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
+                                    }
+                                }
+                            }
+                            // this warp's slice: 32 rows x 32 bytes, 32-byte swizzle (dK, then dV)
+                            const uint32_t dst = sDQw + which * 1024;
+#pragma unroll
+                            for (int q = 0; q < 2; ++q)
+                                st_shared_v4(dst + sw32_off(lane, q), pack_bf16(a[8 * q], a[8 * q + 1]),
+                                             pack_bf16(a[8 * q + 2], a[8 * q + 3]), pack_bf16(a[8 * q + 4], a[8 * q + 5]),
+                                             pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+                        }
                     }
                 }
-            }
-            tc_fence_before();
-            mbar_arrive(&bars->acc_free);  // the next item's first dV, dK may overwrite them
-            if (staged) {
-                // the P area is free: dV of the last tile (its last reader) is done (dq_full)
-                fence_proxy_async_smem();
-                if (warp == 2 && lane == 0) {
-                    bars->store[0] = cur->part.kframe;
-                    bars->store[1] = cur->part.o;
-                    bars->store[2] = cur->w.tile;
-                    bars->store[3] = cur->bh;
+                tc_fence_before();
+                mbar_arrive(&bars->acc_free);  // the next item's first dV, dK may overwrite them
+                if (staged) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        store_warp_slice(p.dk_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OW * g, q4,
+                                         smem + OFF_DQ + warp_slot);
+                        store_warp_slice(p.dv_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OW * g, q4,
+                                         smem + OFF_DQ + warp_slot + 1024);
+                        bulk_commit();
+                    }
                 }
-                mbar_arrive(&bars->stage_full);  // the store warp takes it from here
-                ++SF;
+                done_item(bars, j, true);
+                ++J;
+                if (!has_next) break;
+                ++j;
+                cur = nxt;
+                head_base = static_cast<size_t>(cur->bh) * p.g.n;
+                nq = cur->nq;
+                jj = 0;
             }
-            stage_pending = staged;
-            done_item(bars, j, true);
-            J += nq;
         }
-        if (lane == 0) bulk_wait_read_all();  // this warp's dQ reduces have read their staging
-        if (!F32 && ok && (!stage_pending || wait_all(&bars->stage_free, (SF - 1) & 1))) {
-            if (warp == 2 && lane == 0) bars->store[2] = -1;  // end of the store warp's loop
-            mbar_arrive(&bars->stage_full);
-        }
+        if (lane == 0) bulk_wait_read_all();  // this warp's reduces and stores have read its slot
     }
     tc_fence_before();
     __syncthreads();

@@ -35,7 +35,8 @@ struct FwdParams {
 
 struct BwdParams {
     FrameMaps q, k, v, dout;
-    FrameMaps dk, dv;            // bf16 I/O: dK, dV tile stores (sum used for compacted keys)
+    FrameMaps dk_w, dv_w;        // bf16 I/O: dK, dV in the key frames, 16-column x 32-row boxes
+                                 // (one softmax warp's slice; 32-byte swizzle)
     FrameMaps dq_red;            // fp32 dQ accumulator in the query frames, box 16 columns by
                                  // 32 rows (reduce-add target; nat and col only)
     CUtensorMap dq_direct;       // dQ output (natural frame), box 16 columns by 32 rows: one

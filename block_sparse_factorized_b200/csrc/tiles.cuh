@@ -107,6 +107,27 @@ __device__ __forceinline__ void reduce_warp_f32(const FrameMaps &m, int32_t fr, 
     }
 }
 
+// TMA store of one warp's 32 rows (tile rows 32 q4 .. 32 q4 + 31) x 16 bf16 columns (col0 ..
+// col0 + 15) of key tile t in frame fr (summary offset o).  The maps' boxes are 16 columns by 32
+// rows: {16, 32, 1} natural, {16, min(Rt, 32), max(1, 32 / Rt), 1} grid, {16, min(c, 32),
+// max(1, 32 / c), 1} summary (c a power of two, so the 32 rows are one part of a run or whole
+// runs).  Rows past the tensor (frame padding) are dropped.
+__device__ __forceinline__ void store_warp_slice(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
+                                                 int32_t t, int32_t bh, int32_t col0, int32_t q4, const void *src)
+{
+    const int32_t rho0 = 32 * q4;
+    if (fr == FR_NAT) {
+        tma_store_3d(&m.nat, src, col0, t * TILE + rho0, bh);
+    } else if (fr == FR_COL) {
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
+        const int32_t a0 = fdiv(rho0, g.div_Rt), r0 = rho0 - a0 * g.Rt;
+        tma_store_4d(&m.col, src, col0, rt * TILE + r0, grp * g.cpt + a0, bh);
+    } else {
+        const int32_t kappa = t * TILE + rho0, u = fdiv(kappa, g.div_c), s0 = kappa - u * g.c;
+        tma_store_4d(&m.sum, src, col0, g.l - g.c - o + s0, u, bh);
+    }
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
