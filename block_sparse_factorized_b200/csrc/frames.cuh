@@ -110,7 +110,7 @@ struct SplitRec {
 };
 
 // Longest query run one backward CTA walks; longer runs are split into near-equal chunks.
-constexpr int32_t BWD_CHUNK = 64;
+constexpr int32_t BWD_CHUNK = 48;
 
 ST_HD int32_t imin(int32_t a, int32_t b) { return a < b ? a : b; }
 ST_HD int32_t imax(int32_t a, int32_t b) { return a > b ? a : b; }

@@ -35,7 +35,7 @@ SMALL = [
     Workload("f_single_a2_n512_l32_c4", FIXED, SINGLE_A2, 512, 32, 4, 1, 8),
     Workload("f_merged_n1024_l128_c32", FIXED, MERGED, 1024, 128, 32, 1, 4),
     # long backward items: summary key tile 0 is read by 96 query tiles, more than one backward
-    # chunk (64), so its dK/dV are the sum of two chunks' partials -- also in a merge pass
+    # chunk (48), so its dK/dV are the sum of two chunks' partials -- also in a merge pass
     Workload("f_n12288_l128_c32_long", FIXED, ALTERNATING, 12288, 128, 32, 1, 2),
     Workload("f_merged_n12288_l128_c32_long", FIXED, MERGED, 12288, 128, 32, 1, 1),
     # degenerate sets: c = l (pattern 2 reads every earlier key), c = 128 with three head-2
