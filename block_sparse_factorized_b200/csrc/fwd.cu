@@ -49,8 +49,8 @@ constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 256;            // S: 0..127, O_0: 128..191, O_1: 192..255
 constexpr float RESCALE_LOG2 = 8.0f;           // keep a stale max while it is within 2^8
 
-// Shared-memory plan: the bf16 high and low parts of Q and of each K tile.
-//   Q [, Q_lo] | NST x (K, V [, K_lo]) | P (two 128 x 64 halves: keys 0-63, 64-127) | barriers
+// Shared-memory plan, with the bf16 high and low parts of Q and of each K tile:
+//   Q, Q_lo | NST x (K, V, K_lo) | P (two 128 x 64 halves: keys 0-63, 64-127) | barriers
 // The P area doubles as the (m, l) exchange of the epilogue.
 struct Plan {
     static constexpr uint32_t OFF_Q = 0;

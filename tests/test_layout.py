@@ -92,6 +92,41 @@ def test_argument_errors():
     assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 256
     d = _abi.st_desc_t(1, 2, 256, 64, 2, 0)
     assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 256 + 5 * 2 * 256 * 64 * 2
+    # the split backward's main phase takes dq too (dQ of single-contributor heads is stored there)
+    d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
+    assert lib.st_attn_bwd_main(fake, fake, fake, fake, fake, lay.handle, None, fake, fake, fake, 0,
+                                ctypes.byref(d), None) == 1
+
+
+def test_decode_argument_errors():
+    """The decode step checks its arguments before anything is launched (and needs no upload)."""
+    S, A = bsf.ST_STRIDED, bsf.ST_PER_HEAD_ALTERNATING
+    lib = _abi.load()
+    lay = bsf.Layout(S, A, 2, 256, 16)
+    fake, odd = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
+    # 256 rows of cache -> 4 chunks of 64 keys, 68 floats each, per (batch, head), rounded to 256 B
+    need = lib.st_attn_decode_workspace_bytes(ctypes.byref(d), lay.handle)
+    assert need == 2304
+    ws = ctypes.c_void_p(1 << 24)
+
+    def call(q=fake, pos=100, desc=d, w=ws, wb=need):
+        return lib.st_attn_decode(q, fake, fake, lay.handle, pos, fake, fake, w, wb, ctypes.byref(desc), None)
+
+    assert call(q=None) == 1                      # NULL pointer
+    assert call(pos=-1) == 1 and call(pos=256) == 1   # position outside [0, n)
+    assert call(desc=_abi.st_desc_t(1, 3, 256, 64, 1, 0)) == 1   # heads are not the layout's
+    assert call(desc=_abi.st_desc_t(1, 2, 512, 64, 1, 0)) == 1   # n is not the layout's
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 32, 1, 0)) == 2   # d != 64
+    assert call(q=odd) == 3                       # misaligned
+    assert call(w=None) == 8 and call(wb=need - 1) == 8          # workspace missing / too small
+    keys = np.empty(256, dtype=np.int64)
+    cnt = ctypes.c_int64()
+    kp = keys.ctypes.data_as(ctypes.c_void_p)
+    assert lib.st_decode_row_keys(lay.handle, 2, 0, kp, ctypes.byref(cnt)) == 1   # no head 2
+    assert lib.st_decode_row_keys(lay.handle, 0, 256, kp, ctypes.byref(cnt)) == 1
+    assert lib.st_decode_row_keys(lay.handle, 1, 40, kp, ctypes.byref(cnt)) == 0
+    assert list(keys[:cnt.value]) == [8, 24, 40]  # strided head 2 at i = 40, l = 16
 
 
 def expand_block_row(row_ptr, col_idx, mask_id, masks, qb, B, n):
