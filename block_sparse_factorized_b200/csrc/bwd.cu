@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             auto sQ = [&](int32_t t) { return smem_u32(smem + OFF_Q + (t % NST) * TB); };
             auto sDO = [&](int32_t t) { return smem_u32(smem + OFF_DO + (t % NST) * TB); };
             // Per query tile t the tensor core runs, in order:
-            //   dV += P_t^T dO_t | S_{t+1} | dK += dS_t^T Q_t, dQ_t = dS_t K | dP_{t+1}
+            //   dV += P_t^T dO_t | S_{t+1} | dQ_t = dS_t K, dK += dS_t^T Q_t | dP_{t+1}
             // so that it computes dV_t and S_{t+1} while the softmax warps build dS_t, and dK_t,
             // dQ_t, dP_{t+1} while they drain dQ_t and build P_{t+1}.  An item's first S and dP
             // follow the previous item's last dQ.
@@ -284,16 +284,19 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                         break;
                     tc_fence_after();
                     const uint32_t sK = smem_u32(smem + OFF_K + ks * TB);
-                    // dK += dS^T Q (as dV), dQ = dS K: A = dS K-major (two 64-key halves), B = K MN-major
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + kk * 2048, TB, 1024),
-                                    desc_sw128(sQ(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
+                    // dQ = dS K (A = dS K-major, two 64-key halves; B = K MN-major), signalled at once
+                    // so that the drain can start, then dK += dS^T Q (as dV); on an item's last tile
+                    // dq_full waits for dK too, since the epilogue reads it
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (kk >> 2) * TB + (kk & 3) * 32, 16, 1024),
                                     desc_sw128(sK + kk * 2048, TB, 1024), id_kt, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->dq_full);   // also: dK, dV of the item complete on its last tile
+                    if (!last) mma_commit(&bars->dq_full);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + kk * 2048, TB, 1024),
+                                    desc_sw128(sQ(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
+                    if (last) mma_commit(&bars->dq_full);  // also: dK, dV of the item complete
                     mma_commit(&bars->qdo_empty[t % NST]);
                     if (last) {
                         mma_commit(&bars->kv_empty[ks]);  // K and V of this item are no longer read
