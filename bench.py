@@ -356,8 +356,10 @@ def run_ours(args, rank, world, local):
     ms_local = statistics.mean(t_step)
     ms = max_over_ranks(ms_local, world, device)
     value = flops * world / (ms / 1e3) / 1e12
-    # fwd per pass; bwd: prepare, the main kernel per pass, a summing pass per split pass, convert
-    launches_per_step = 2 * info["passes"] + 2 + info["split_passes"]
+    # fwd per pass; bwd: prepare, the main kernel per pass, a summing pass per split pass, and
+    # the convert pass unless every head's dQ is stored by the main kernel
+    launches_per_step = (2 * info["passes"] + 1 + info["split_passes"] +
+                         (1 if info["dq_direct_heads"] < w.heads else 0))
     peaks = measured_peaks()
     main_ms = statistics.mean(t_main)
     achieved = bwd_flops / (main_ms / 1e3) / 1e12
