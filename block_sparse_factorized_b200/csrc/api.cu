@@ -517,8 +517,11 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     p.bh = static_cast<int32_t>(desc->batch * desc->heads);
     p.heads = static_cast<int32_t>(desc->heads);
     p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
-    const int32_t nsplit = static_cast<int32_t>((most + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
-    return st::launch_decode(p, nsplit, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+    const int64_t nsplit = (most + st::DEC_CHUNK - 1) / st::DEC_CHUNK;
+    if (nsplit > 65535) return ST_ERR_UNSUPPORTED;  // grid dimension y: a row with over 4 M allowed keys
+    return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, stream) == cudaSuccess
+               ? ST_OK
+               : ST_ERR_CUDA;
 }
 
 st_status_t st_decode_row_keys(const st_layout_t *layout, int32_t head, int64_t pos, int64_t *keys, int64_t *count)

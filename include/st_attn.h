@@ -248,7 +248,8 @@ ST_API st_status_t st_attn_bwd_noalloc(const void *q, const void *k, const void 
  * desc is the full-sequence descriptor (its n is the cache capacity).  The layout need not be
  * uploaded: the kernels read only the per-head set kinds, passed by value.  Errors:
  * ST_ERR_INVALID_ARG (NULL pointers, pos outside [0, n), heads or n not the layout's),
- * ST_ERR_UNSUPPORTED (d != 64, more than 64 heads), ST_ERR_ALIGNMENT, ST_ERR_WORKSPACE,
+ * ST_ERR_UNSUPPORTED (d != 64, more than 64 heads, a row with over 4,194,240 allowed keys),
+ * ST_ERR_ALIGNMENT, ST_ERR_WORKSPACE,
  * ST_ERR_CUDA. */
 ST_API size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout);
 ST_API st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache,
