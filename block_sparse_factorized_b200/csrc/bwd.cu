@@ -627,18 +627,6 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     }
 }
 
-int sm_count()
-{
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <bool F32>
 cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
 {

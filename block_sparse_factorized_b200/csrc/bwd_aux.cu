@@ -243,19 +243,22 @@ __global__ void __launch_bounds__(512) split_finish_kernel(const SplitFinishPara
     }
 }
 
+}  // namespace
+
 int sm_count()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    constexpr int MAXDEV = 64;
+    static int count[MAXDEV] = {};  // per device, filled on first use
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+    if (dev >= MAXDEV) dev = MAXDEV - 1;
+    if (count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        count[dev] = n;
     }
-    return n;
+    return count[dev];
 }
-
-}  // namespace
 
 int blocks_for(int64_t work_units)
 {

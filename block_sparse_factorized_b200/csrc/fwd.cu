@@ -536,18 +536,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
-int sm_count()
-{
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 cudaError_t launch_fwd_split(const FwdParams &p, cudaStream_t s)
 {
     static bool configured = false;

@@ -479,10 +479,7 @@ cudaError_t launch_fwd_bf16(const FwdParams &p, cudaStream_t s)
     }
     const int64_t units = static_cast<int64_t>(p.nitems) * p.batch;
     if (units == 0) return cudaSuccess;
-    int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * CTAS_PER_SM;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * CTAS_PER_SM;
     fwd_bf16_kernel<<<static_cast<unsigned>(units < cap ? units : cap), THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
 }

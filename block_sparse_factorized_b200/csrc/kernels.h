@@ -100,6 +100,9 @@ struct SplitParams {
     int64_t elems;
 };
 
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count();
+
 cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s);
 cudaError_t launch_fwd_bf16(const FwdParams &p, cudaStream_t s);
 cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
