@@ -64,3 +64,25 @@ def test_reference_arm_nonzero_ranks_exit_quietly():
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
                        timeout=300, cwd=ROOT, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_headline_flop_and_byte_counts():
+    """The metric's FLOP count at the headline workload: 10,368 active 128 x 128 tile pairs (4 x 96
+    same-block + 4 x 1,200 summary per batch element, x 2), 4 d FLOPs per score entry in the
+    forward and 2.5 times that in the backward; the algorithmic bytes count each tensor once
+    (a summary head reads n / l * c key rows)."""
+    import block_sparse_factorized_b200 as bsf
+    from workloads import WORKLOADS
+    w = WORKLOADS["fixed_n12288_l128_c32"]
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c)
+    flops, bwd_flops, useful = bench.step_flops(w, lay.info())
+    pairs = 2 * (4 * 96 + 4 * 1200)
+    assert pairs == 10368
+    assert flops == pairs * 128 * 128 * 4 * 64 * 3.5
+    assert bwd_flops == pairs * 128 * 128 * 4 * 64 * 2.5
+    assert useful == 78673920 * 2 * 4 * 64 * 3.5  # allowed (i, j) pairs only
+    fwd_b, bwd_b = bench.step_bytes(w, lay)
+    rows, row = 2 * 8 * 12288, 128
+    used = 2 * (4 * 12288 + 4 * 96 * 32)  # K/V rows read: 4 full heads + 4 summary heads
+    assert fwd_b == 2 * rows * row + 2 * used * row + rows * 4
+    assert bwd_b == fwd_b + rows * row + rows * 4 + 3 * rows * row
