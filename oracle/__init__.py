@@ -52,11 +52,11 @@ def _L():
         lib.oracle_set_counts.argtypes = [i32, i64, i64, i64, i64, p]
         lib.oracle_head_kinds.argtypes = [i32, i32, i32, i64, i64, i64, p, p]
         lib.oracle_head_kinds.restype = i32
-        common = [p, p, p, i64, i64, i64, i64, p, p, i64, i64]
+        common = [p, p, p, i64, i64, i64, i64, i64, p, p, i64, i64]
         lib.oracle_fwd.argtypes = common + [p, p]
         lib.oracle_fwd_rows.argtypes = common + [i64, p, p, p]
         lib.oracle_decode.argtypes = common + [i64, p, p]
-        bcommon = [p, p, p, p, i64, i64, i64, i64, p, p, i64, i64]
+        bcommon = [p, p, p, p, i64, i64, i64, i64, i64, p, p, i64, i64]
         lib.oracle_bwd.argtypes = bcommon + [p, p, p]
         lib.oracle_bwd_rows.argtypes = bcommon + [i64, p, p, p, p]
         lib.oracle_bwd_keys.argtypes = bcommon + [i64, p, p, p]
@@ -98,8 +98,18 @@ def head_kinds(family: int, head_mode: int, num_heads: int, l: int, c: int = 0, 
     return kind, off
 
 
+def _dims(q, k, v, do=None):
+    """(B, H, n, d, e): q and k are [B, H, n, d], v (and do) [B, H, n, e]."""
+    B, H, n, d = q.shape
+    e = v.shape[-1]
+    if k.shape != (B, H, n, d) or v.shape != (B, H, n, e) or (do is not None and do.shape != v.shape):
+        raise ValueError("q, k must be [B, H, n, d] and v, dO [B, H, n, e]")
+    return B, H, n, d, e
+
+
 class Problem:
-    """Per-head set kinds and offsets for one pattern; shapes are [B, H, n, d]."""
+    """Per-head set kinds and offsets for one pattern.  Q and K are [B, H, n, d]; V, O and dO are
+    [B, H, n, e] (e = d unless the query-key width is reduced)."""
 
     def __init__(self, family: int, head_mode: int, num_heads: int, l: int, c: int = 0,
                  step: int = 0):
@@ -116,55 +126,56 @@ class Problem:
 
     def fwd(self, q, k, v):
         q, k, v = _f64(q), _f64(k), _f64(v)
-        B, H, n, d = q.shape
-        o = np.empty_like(q)
+        B, H, n, d, e = _dims(q, k, v)
+        o = np.empty_like(v)
         lse = np.empty((B, H, n), dtype=np.float64)
-        _L().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, _ptr(self.kind), _ptr(self.off),
+        _L().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, e, _ptr(self.kind), _ptr(self.off),
                         self.l, self.c, _ptr(o), _ptr(lse))
         return o, lse
 
     def fwd_rows(self, q, k, v, rows):
         """rows: flat indices (b*H + h)*n + i."""
         q, k, v = _f64(q), _f64(k), _f64(v)
-        B, H, n, d = q.shape
+        B, H, n, d, e = _dims(q, k, v)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
-        o = np.empty((len(rows), d), dtype=np.float64)
+        o = np.empty((len(rows), e), dtype=np.float64)
         lse = np.empty(len(rows), dtype=np.float64)
-        _L().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, _ptr(self.kind),
+        _L().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, e, _ptr(self.kind),
                              _ptr(self.off), self.l, self.c, len(rows), _ptr(rows), _ptr(o),
                              _ptr(lse))
         return o, lse
 
     def decode(self, q, k, v, pos):
         """One query row per (batch, head) at position pos against the cache rows 0..pos.
-        q: [B, H, d]; k, v: [B, H, n, d].  Returns o [B, H, d], lse [B, H]."""
+        q: [B, H, d]; k: [B, H, n, d]; v: [B, H, n, e].  Returns o [B, H, e], lse [B, H]."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, n, d = k.shape
-        if q.shape != (B, H, d) or not 0 <= pos < n:
-            raise ValueError("q must be [B, H, d] and 0 <= pos < n")
-        o = np.empty_like(q)
+        e = v.shape[-1]
+        if q.shape != (B, H, d) or v.shape != (B, H, n, e) or not 0 <= pos < n:
+            raise ValueError("q must be [B, H, d], v [B, H, n, e] and 0 <= pos < n")
+        o = np.empty((B, H, e), dtype=np.float64)
         lse = np.empty((B, H), dtype=np.float64)
-        _L().oracle_decode(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, _ptr(self.kind), _ptr(self.off),
+        _L().oracle_decode(_ptr(q), _ptr(k), _ptr(v), B, H, n, d, e, _ptr(self.kind), _ptr(self.off),
                            self.l, self.c, int(pos), _ptr(o), _ptr(lse))
         return o, lse
 
     def bwd(self, q, k, v, do):
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
-        B, H, n, d = q.shape
-        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
-        _L().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, _ptr(self.kind),
+        B, H, n, d, e = _dims(q, k, v, do)
+        dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+        _L().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, e, _ptr(self.kind),
                         _ptr(self.off), self.l, self.c, _ptr(dq), _ptr(dk), _ptr(dv))
         return dq, dk, dv
 
     def bwd_rows(self, q, k, v, do, rows):
         """dQ (and lse, D) for flat query rows."""
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
-        B, H, n, d = q.shape
+        B, H, n, d, e = _dims(q, k, v, do)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         dq = np.empty((len(rows), d), dtype=np.float64)
         lse = np.empty(len(rows), dtype=np.float64)
         D = np.empty(len(rows), dtype=np.float64)
-        _L().oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, _ptr(self.kind),
+        _L().oracle_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, e, _ptr(self.kind),
                              _ptr(self.off), self.l, self.c, len(rows), _ptr(rows), _ptr(dq),
                              _ptr(lse), _ptr(D))
         return dq, lse, D
@@ -172,11 +183,11 @@ class Problem:
     def bwd_keys(self, q, k, v, do, keys):
         """dK and dV for flat key rows."""
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
-        B, H, n, d = q.shape
+        B, H, n, d, e = _dims(q, k, v, do)
         keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
         dk = np.empty((len(keys), d), dtype=np.float64)
-        dv = np.empty((len(keys), d), dtype=np.float64)
-        _L().oracle_bwd_keys(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, _ptr(self.kind),
+        dv = np.empty((len(keys), e), dtype=np.float64)
+        _L().oracle_bwd_keys(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, H, n, d, e, _ptr(self.kind),
                              _ptr(self.off), self.l, self.c, len(keys), _ptr(keys), _ptr(dk),
                              _ptr(dv))
         return dk, dv

@@ -17,7 +17,8 @@
  * Everything is the plain definition written out: each allowed set is found by scanning
  * j = 0..i with the page predicate; scores, a two-pass softmax and the output follow; the
  * gradients are ordinary calculus of that definition (no recompute trick, no blocking, no online
- * softmax).  All arithmetic is in double precision.  Readings taken where the pages are silent or
+ * softmax).  All arithmetic is in double precision.  Query and key rows have width d, value,
+ * output and output-gradient rows width e (e = d unless the query-key projection is narrower).  Readings taken where the pages are silent or
  * garbled are listed next to each function.
  *
  * Set kinds (one per head):
@@ -117,15 +118,17 @@ int oracle_head_kinds(int family, int head_mode, int num_heads, int64_t l, int64
  * two-pass softmax  m = max_j S_ij, Z = sum_j exp(S_ij - m), P_ij = exp(S_ij - m) / Z, and
  * O_i = sum_j P_ij v_j, lse_i = m + ln Z ([G] §02).  Reading for a row with no allowed key
  * ([G] §02 warns such a row has no softmax): O_i = 0 and lse_i = -inf.
- * qi is the query row; kh, vh point at the (batch, head) slab of n x d values.  set and s are
+ * Widths: d is the width of the query and key rows (the dot product, hence the 1/sqrt(d) scale),
+ * e the width of the value rows and of O.  e = d except with half-size query-key projections
+ * ([R] §4.5: the CIFAR-10 model halves its QK projection, so d = e / 2 there).
+ * qi is the query row; kh (n x d) and vh (n x e) point at the (batch, head) slabs.  set and s are
  * scratch of n. */
-static void fwd_row(const double *qi, const double *kh, const double *vh, int64_t n, int64_t d,
+static void fwd_row(const double *qi, const double *kh, const double *vh, int64_t d, int64_t e,
                     int kind, int64_t l, int64_t c, int64_t o, int64_t i, int64_t *set, double *s,
                     double *orow, double *lse)
 {
-    (void)n;
     int64_t cnt = oracle_row_set(kind, i, l, c, o, set);
-    for (int64_t t = 0; t < d; ++t) orow[t] = 0.0;
+    for (int64_t t = 0; t < e; ++t) orow[t] = 0.0;
     if (cnt == 0) { *lse = -INFINITY; return; }
     const double scale = 1.0 / sqrt((double)d);
     double m = -INFINITY;
@@ -140,15 +143,16 @@ static void fwd_row(const double *qi, const double *kh, const double *vh, int64_
     for (int64_t a = 0; a < cnt; ++a) z += exp(s[a] - m);
     for (int64_t a = 0; a < cnt; ++a) {
         const double p = exp(s[a] - m) / z;
-        const double *vj = vh + set[a] * d;
-        for (int64_t t = 0; t < d; ++t) orow[t] += p * vj[t];
+        const double *vj = vh + set[a] * e;
+        for (int64_t t = 0; t < e; ++t) orow[t] += p * vj[t];
     }
     *lse = m + log(z);
 }
 
+/* Full forward.  q, k: B x H x n x d; v, o: B x H x n x e; lse: B x H x n. */
 void oracle_fwd(const double *q, const double *k, const double *v, int64_t B, int64_t H, int64_t n,
-                int64_t d, const int *kind, const int64_t *off, int64_t l, int64_t c, double *o,
-                double *lse)
+                int64_t d, int64_t e, const int *kind, const int64_t *off, int64_t l, int64_t c,
+                double *o, double *lse)
 {
 #pragma omp parallel
     {
@@ -157,18 +161,18 @@ void oracle_fwd(const double *q, const double *k, const double *v, int64_t B, in
 #pragma omp for schedule(dynamic, 32)
         for (int64_t r = 0; r < B * H * n; ++r) {
             const int64_t bh = r / n, i = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            fwd_row(q + base + (size_t)i * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], i,
-                    set, s, o + (size_t)r * (size_t)d, lse + r);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            fwd_row(q + bq + (size_t)i * (size_t)d, k + bq, v + bv, d, e, kind[h], l, c, off[h], i,
+                    set, s, o + (size_t)r * (size_t)e, lse + r);
         }
         free(set);
         free(s);
     }
 }
 
-/* Forward for a chosen list of flat rows r = (b*H + h)*n + i; o_rows is nrows x d. */
+/* Forward for a chosen list of flat rows r = (b*H + h)*n + i; o_rows is nrows x e. */
 void oracle_fwd_rows(const double *q, const double *k, const double *v, int64_t B, int64_t H,
-                     int64_t n, int64_t d, const int *kind, const int64_t *off, int64_t l,
+                     int64_t n, int64_t d, int64_t e, const int *kind, const int64_t *off, int64_t l,
                      int64_t c, int64_t nrows, const int64_t *rows, double *o_rows,
                      double *lse_rows)
 {
@@ -180,9 +184,9 @@ void oracle_fwd_rows(const double *q, const double *k, const double *v, int64_t 
 #pragma omp for schedule(dynamic, 1)
         for (int64_t a = 0; a < nrows; ++a) {
             const int64_t r = rows[a], bh = r / n, i = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            fwd_row(q + base + (size_t)i * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], i,
-                    set, s, o_rows + (size_t)a * (size_t)d, lse_rows + a);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            fwd_row(q + bq + (size_t)i * (size_t)d, k + bq, v + bv, d, e, kind[h], l, c, off[h], i,
+                    set, s, o_rows + (size_t)a * (size_t)e, lse_rows + a);
         }
         free(set);
         free(s);
@@ -193,11 +197,11 @@ void oracle_fwd_rows(const double *q, const double *k, const double *v, int64_t 
  * values of rows 0..pos (the sampling setting of [R] §2/§3, where each generated position attends
  * to its allowed set among the positions already produced).  By the definition of A(pos) (a
  * subset of {j <= pos}) this is exactly row pos of the forward pass: the same fwd_row, with the
- * query taken from q[b, h] instead of Q[b, h, pos].  q, o: B x H x d; k, v: B x H x n x d (rows
- * past pos are never read); lse: B x H. */
+ * query taken from q[b, h] instead of Q[b, h, pos].  q: B x H x d; k: B x H x n x d; v:
+ * B x H x n x e (rows past pos are never read); o: B x H x e; lse: B x H. */
 void oracle_decode(const double *q, const double *k, const double *v, int64_t B, int64_t H, int64_t n,
-                   int64_t d, const int *kind, const int64_t *off, int64_t l, int64_t c, int64_t pos,
-                   double *o, double *lse)
+                   int64_t d, int64_t e, const int *kind, const int64_t *off, int64_t l, int64_t c,
+                   int64_t pos, double *o, double *lse)
 {
 #pragma omp parallel
     {
@@ -206,9 +210,9 @@ void oracle_decode(const double *q, const double *k, const double *v, int64_t B,
 #pragma omp for schedule(dynamic, 1)
         for (int64_t bh = 0; bh < B * H; ++bh) {
             const int64_t h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            fwd_row(q + (size_t)bh * (size_t)d, k + base, v + base, n, d, kind[h], l, c, off[h], pos, set, s,
-                    o + (size_t)bh * (size_t)d, lse + bh);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            fwd_row(q + (size_t)bh * (size_t)d, k + bq, v + bv, d, e, kind[h], l, c, off[h], pos, set,
+                    s, o + (size_t)bh * (size_t)e, lse + bh);
         }
         free(set);
         free(s);
@@ -227,22 +231,24 @@ void oracle_decode(const double *q, const double *k, const double *v, int64_t B,
  * [R] §3.4 recomputes attention in the backward pass instead of storing it; that is a
  * memory/time trade with no effect on these values, so the oracle simply evaluates them. */
 
-/* Row quantities of query i: lse_i, D_i and (if dqrow != NULL) dQ_i. */
+/* Row quantities of query i: lse_i, D_i and (if dqrow != NULL) dQ_i.  qh, kh, dqrow have rows of
+ * width d; vh, doh rows of width e (see fwd_row). */
 static void bwd_row(const double *qh, const double *kh, const double *vh, const double *doh,
-                    int64_t d, int kind, int64_t l, int64_t c, int64_t o, int64_t i, int64_t *set,
-                    double *s, double *dp, double *lse_out, double *D_out, double *dqrow)
+                    int64_t d, int64_t e, int kind, int64_t l, int64_t c, int64_t o, int64_t i,
+                    int64_t *set, double *s, double *dp, double *lse_out, double *D_out, double *dqrow)
 {
     const double scale = 1.0 / sqrt((double)d);
     int64_t cnt = oracle_row_set(kind, i, l, c, o, set);
     if (dqrow)
         for (int64_t t = 0; t < d; ++t) dqrow[t] = 0.0;
     if (cnt == 0) { *lse_out = -INFINITY; *D_out = 0.0; return; }
+    const double *qi = qh + i * d, *doi = doh + i * e;
     double m = -INFINITY;
     for (int64_t a = 0; a < cnt; ++a) {
-        const double *qi = qh + i * d, *kj = kh + set[a] * d, *vj = vh + set[a] * d,
-                     *doi = doh + i * d;
+        const double *kj = kh + set[a] * d, *vj = vh + set[a] * e;
         double acc = 0.0, accp = 0.0;
-        for (int64_t t = 0; t < d; ++t) { acc += qi[t] * kj[t]; accp += doi[t] * vj[t]; }
+        for (int64_t t = 0; t < d; ++t) acc += qi[t] * kj[t];
+        for (int64_t t = 0; t < e; ++t) accp += doi[t] * vj[t];
         s[a] = acc * scale;
         dp[a] = accp;
         if (s[a] > m) m = s[a];
@@ -262,31 +268,33 @@ static void bwd_row(const double *qh, const double *kh, const double *vh, const 
     *D_out = D;
 }
 
-/* Key quantities of key j given lse and D of every row of the (batch, head). */
+/* Key quantities of key j given lse and D of every row of the (batch, head): dK_j (width d) and
+ * dV_j (width e). */
 static void bwd_key(const double *qh, const double *kh, const double *vh, const double *doh,
-                    int64_t n, int64_t d, int kind, int64_t l, int64_t c, int64_t o, int64_t j,
-                    const double *lse, const double *D, double *dkrow, double *dvrow)
+                    int64_t n, int64_t d, int64_t e, int kind, int64_t l, int64_t c, int64_t o,
+                    int64_t j, const double *lse, const double *D, double *dkrow, double *dvrow)
 {
     const double scale = 1.0 / sqrt((double)d);
-    for (int64_t t = 0; t < d; ++t) { dkrow[t] = 0.0; dvrow[t] = 0.0; }
-    const double *kj = kh + j * d, *vj = vh + j * d;
+    for (int64_t t = 0; t < d; ++t) dkrow[t] = 0.0;
+    for (int64_t t = 0; t < e; ++t) dvrow[t] = 0.0;
+    const double *kj = kh + j * d, *vj = vh + j * e;
     for (int64_t i = j; i < n; ++i) {
         if (!oracle_allowed(kind, i, j, l, c, o)) continue;
-        const double *qi = qh + i * d, *doi = doh + i * d;
+        const double *qi = qh + i * d, *doi = doh + i * e;
         double acc = 0.0, accp = 0.0;
-        for (int64_t t = 0; t < d; ++t) { acc += qi[t] * kj[t]; accp += doi[t] * vj[t]; }
+        for (int64_t t = 0; t < d; ++t) acc += qi[t] * kj[t];
+        for (int64_t t = 0; t < e; ++t) accp += doi[t] * vj[t];
         const double p = exp(acc * scale - lse[i]);
         const double ds = p * (accp - D[i]);
-        for (int64_t t = 0; t < d; ++t) {
-            dvrow[t] += p * doi[t];
-            dkrow[t] += ds * qi[t] * scale;
-        }
+        for (int64_t t = 0; t < e; ++t) dvrow[t] += p * doi[t];
+        for (int64_t t = 0; t < d; ++t) dkrow[t] += ds * qi[t] * scale;
     }
 }
 
+/* Full backward.  q, k, dq, dk: B x H x n x d; v, dout, dv: B x H x n x e. */
 void oracle_bwd(const double *q, const double *k, const double *v, const double *dout, int64_t B,
-                int64_t H, int64_t n, int64_t d, const int *kind, const int64_t *off, int64_t l,
-                int64_t c, double *dq, double *dk, double *dv)
+                int64_t H, int64_t n, int64_t d, int64_t e, const int *kind, const int64_t *off,
+                int64_t l, int64_t c, double *dq, double *dk, double *dv)
 {
     const int64_t rows = B * H * n;
     double *lse = (double *)malloc(sizeof(double) * (size_t)rows);
@@ -299,17 +307,16 @@ void oracle_bwd(const double *q, const double *k, const double *v, const double 
 #pragma omp for schedule(dynamic, 32)
         for (int64_t r = 0; r < rows; ++r) {
             const int64_t bh = r / n, i = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            bwd_row(q + base, k + base, v + base, dout + base, d, kind[h], l, c, off[h], i, set,
-                    s, dp, lse + r, D + r, dq + (size_t)r * (size_t)d);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            bwd_row(q + bq, k + bq, v + bv, dout + bv, d, e, kind[h], l, c, off[h], i, set, s, dp,
+                    lse + r, D + r, dq + (size_t)r * (size_t)d);
         }
 #pragma omp for schedule(dynamic, 32)
         for (int64_t r = 0; r < rows; ++r) {
             const int64_t bh = r / n, j = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            bwd_key(q + base, k + base, v + base, dout + base, n, d, kind[h], l, c, off[h], j,
-                    lse + bh * n, D + bh * n, dk + (size_t)r * (size_t)d,
-                    dv + (size_t)r * (size_t)d);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            bwd_key(q + bq, k + bq, v + bv, dout + bv, n, d, e, kind[h], l, c, off[h], j,
+                    lse + bh * n, D + bh * n, dk + (size_t)r * (size_t)d, dv + (size_t)r * (size_t)e);
         }
         free(set);
         free(s);
@@ -319,9 +326,9 @@ void oracle_bwd(const double *q, const double *k, const double *v, const double 
     free(D);
 }
 
-/* dQ for a chosen list of flat query rows; also returns each row's lse and D. */
+/* dQ for a chosen list of flat query rows (nrows x d); also returns each row's lse and D. */
 void oracle_bwd_rows(const double *q, const double *k, const double *v, const double *dout,
-                     int64_t B, int64_t H, int64_t n, int64_t d, const int *kind,
+                     int64_t B, int64_t H, int64_t n, int64_t d, int64_t e, const int *kind,
                      const int64_t *off, int64_t l, int64_t c, int64_t nrows, const int64_t *rows,
                      double *dq_rows, double *lse_rows, double *D_rows)
 {
@@ -334,9 +341,9 @@ void oracle_bwd_rows(const double *q, const double *k, const double *v, const do
 #pragma omp for schedule(dynamic, 1)
         for (int64_t a = 0; a < nrows; ++a) {
             const int64_t r = rows[a], bh = r / n, i = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            bwd_row(q + base, k + base, v + base, dout + base, d, kind[h], l, c, off[h], i, set,
-                    s, dp, lse_rows + a, D_rows + a, dq_rows + (size_t)a * (size_t)d);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            bwd_row(q + bq, k + bq, v + bv, dout + bv, d, e, kind[h], l, c, off[h], i, set, s, dp,
+                    lse_rows + a, D_rows + a, dq_rows + (size_t)a * (size_t)d);
         }
         free(set);
         free(s);
@@ -344,10 +351,11 @@ void oracle_bwd_rows(const double *q, const double *k, const double *v, const do
     }
 }
 
-/* dK and dV for a chosen list of flat key rows r = (b*H + h)*n + j.  The lse and D of every row
- * of each (batch, head) that owns a chosen key are evaluated first (plain row formulas). */
+/* dK (nkeys x d) and dV (nkeys x e) for a chosen list of flat key rows r = (b*H + h)*n + j.  The
+ * lse and D of every row of each (batch, head) that owns a chosen key are evaluated first (plain
+ * row formulas). */
 void oracle_bwd_keys(const double *q, const double *k, const double *v, const double *dout,
-                     int64_t B, int64_t H, int64_t n, int64_t d, const int *kind,
+                     int64_t B, int64_t H, int64_t n, int64_t d, int64_t e, const int *kind,
                      const int64_t *off, int64_t l, int64_t c, int64_t nkeys, const int64_t *keys,
                      double *dk_rows, double *dv_rows)
 {
@@ -365,17 +373,17 @@ void oracle_bwd_keys(const double *q, const double *k, const double *v, const do
         for (int64_t r = 0; r < nbh * n; ++r) {
             const int64_t bh = r / n, i = r % n, h = bh % H;
             if (!need[bh]) continue;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            bwd_row(q + base, k + base, v + base, dout + base, d, kind[h], l, c, off[h], i, set,
-                    s, dp, lse + r, D + r, NULL);
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            bwd_row(q + bq, k + bq, v + bv, dout + bv, d, e, kind[h], l, c, off[h], i, set, s, dp,
+                    lse + r, D + r, NULL);
         }
 #pragma omp for schedule(dynamic, 1)
         for (int64_t a = 0; a < nkeys; ++a) {
             const int64_t r = keys[a], bh = r / n, j = r % n, h = bh % H;
-            const size_t base = (size_t)bh * (size_t)n * (size_t)d;
-            bwd_key(q + base, k + base, v + base, dout + base, n, d, kind[h], l, c, off[h], j,
+            const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
+            bwd_key(q + bq, k + bq, v + bv, dout + bv, n, d, e, kind[h], l, c, off[h], j,
                     lse + bh * n, D + bh * n, dk_rows + (size_t)a * (size_t)d,
-                    dv_rows + (size_t)a * (size_t)d);
+                    dv_rows + (size_t)a * (size_t)e);
         }
         free(set);
         free(s);

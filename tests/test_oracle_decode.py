@@ -71,3 +71,18 @@ def test_decode_zero_query_is_uniform(kind):
     keys = oracle.row_set(kind, pos, l, c, 1 if kind in (FA2, FU) else 0)
     np.testing.assert_allclose(lse[0, 0], math.log(len(keys)), rtol=0, atol=1e-14)
     np.testing.assert_allclose(o[0, 0], v[0, 0, keys].mean(0), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("d,e", [(32, 32), (64, 128), (128, 128)])
+def test_decode_equals_forward_row_widths(d, e):
+    """Query-key rows of width d, value rows of width e: the decode row is still row pos of the
+    forward (whose widths are pinned in test_oracle_math)."""
+    B, H, n, l, c, pos = 1, 6, 40, 8, 3, 37
+    k, v = rand((B, H, n, d), 13), rand((B, H, n, e), 14)
+    q = rand((B, H, n, d), 15)
+    p = oracle.Problem.from_kinds(list(ALL), [0, 0, 0, 0, 2, 2], l, c)
+    O, lse = p.fwd(q, k, v)
+    o, l_ = p.decode(q[:, :, pos].copy(), k, v, pos)
+    assert o.shape == (B, H, e)
+    np.testing.assert_array_equal(o, O[:, :, pos])
+    np.testing.assert_array_equal(l_, lse[:, :, pos])

@@ -26,8 +26,16 @@ MUTATIONS = {
                           "case K_FA2: return (j % l) >= l - c + o && (j % l) <= l - 1 + o;"),
     "scale_dropped": ("const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;"),
     "softmax_unnormalised": ("const double p = exp(s[a] - m) / z;", "const double p = exp(s[a] - m);"),
-    "values_read_from_keys": ("const double *vj = vh + set[a] * d;\n        for (int64_t t = 0; t < d; ++t) orow[t]",
-                              "const double *vj = kh + set[a] * d;\n        for (int64_t t = 0; t < d; ++t) orow[t]"),
+    "values_read_from_keys": ("const double *vj = vh + set[a] * e;\n        for (int64_t t = 0; t < e; ++t) orow[t]",
+                              "const double *vj = kh + set[a] * e;\n        for (int64_t t = 0; t < e; ++t) orow[t]"),
+    # the two widths confused: the score scaled by the value width, value rows stepped by the
+    # query-key width, dO rows stepped by the query-key width
+    "scale_uses_value_width": ("const double scale = 1.0 / sqrt((double)d);",
+                               "const double scale = 1.0 / sqrt((double)e);"),
+    "value_rows_at_qk_width": ("const double *vj = vh + set[a] * e;\n        for (int64_t t = 0; t < e; ++t) orow[t]",
+                               "const double *vj = vh + set[a] * d;\n        for (int64_t t = 0; t < e; ++t) orow[t]"),
+    "dO_rows_at_qk_width": ("const double *qi = qh + i * d, *doi = doh + i * e;",
+                            "const double *qi = qh + i * d, *doi = doh + i * d;"),
     "lse_missing_max": ("*lse = m + log(z);", "*lse = log(z);"),
     "dS_sign": ("const double ds = p * (accp - D[i]);", "const double ds = p * (accp + D[i]);"),
     "dK_scale_dropped": ("dkrow[t] += ds * qi[t] * scale;", "dkrow[t] += ds * qi[t];"),
