@@ -118,7 +118,9 @@ class Layout:
             h.value = None  # (at interpreter exit the ctypes module may already be gone)
 
 
-def _desc(q: torch.Tensor) -> _abi.st_desc_t:
+def _desc(q: torch.Tensor, v: torch.Tensor | None = None) -> _abi.st_desc_t:
+    """Descriptor of a call: q is [batch, heads, n, d]; v (if given) [batch, heads, n, dv].  The
+    value width is sent as 0 ("same as d") when the two widths agree."""
     if q.dim() != 4:
         raise ValueError("expected [batch, heads, n, d] tensors")
     B, H, n, d = q.shape
@@ -128,18 +130,27 @@ def _desc(q: torch.Tensor) -> _abi.st_desc_t:
         dt = ST_FP32
     else:
         raise TypeError(f"unsupported dtype {q.dtype}")
-    return _abi.st_desc_t(B, H, n, d, dt, 0)
+    dv = 0 if v is None or v.shape[-1] == d else int(v.shape[-1])
+    return _abi.st_desc_t(B, H, n, d, dt, dv)
 
 
-def _check_tensors(*ts):
-    ref = ts[0]
-    for t in ts:
+def _check_tensors(qk, vo=()):
+    """qk: tensors of query-key width ([B, H, n, d]: q, k, dq, dk); vo: tensors of value width
+    ([B, H, n, dv]: v, o, dO, dv).  All contiguous CUDA tensors of one dtype and device."""
+    ref = qk[0]
+    for t in (*qk, *vo):
         if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors (no CPU path exists)")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
-        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
-            raise ValueError("q, k, v (and o, dO) must share shape, dtype and device")
+        if t.dim() != 4 or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("tensors must be [B, H, n, width] of one dtype and device")
+    for t in qk:
+        if t.shape != ref.shape:
+            raise ValueError("q and k (and dq, dk) must share one shape [B, H, n, d]")
+    for t in vo:
+        if t.shape[:3] != ref.shape[:3] or t.shape[3] != vo[0].shape[3]:
+            raise ValueError("v, o, dO (and dv) must share one shape [B, H, n, dv]")
 
 
 def _ptr(t):
@@ -158,11 +169,11 @@ def st_attn_bwd_workspace_bytes(q: torch.Tensor, layout: Layout) -> int:
 
 def st_attn_fwd(q, k, v, layout: Layout, o=None, lse=None, workspace=None, stream=None):
     """O and lse ([B, H, n] fp32, natural log) of factorized sparse attention."""
-    _check_tensors(q, k, v)
-    desc = _desc(q)
+    _check_tensors((q, k), (v,) if o is None else (v, o))
+    desc = _desc(q, v)
     B, H, n, _ = q.shape
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty_like(v)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
     ws = int(layout._lib.st_attn_fwd_workspace_bytes(_c.byref(desc), layout.handle))
@@ -178,14 +189,14 @@ def st_attn_fwd(q, k, v, layout: Layout, o=None, lse=None, workspace=None, strea
 def st_attn_bwd(q, k, v, o, lse, do, layout: Layout, dq=None, dk=None, dv=None, workspace=None,
                 stream=None):
     """dQ, dK, dV of factorized sparse attention (recomputing P from the saved lse)."""
-    _check_tensors(q, k, v, o, do)
-    desc = _desc(q)
+    _check_tensors((q, k), (v, o, do))
+    desc = _desc(q, v)
     if dq is None:
         dq = torch.empty_like(q)
     if dk is None:
-        dk = torch.empty_like(q)
+        dk = torch.empty_like(k)
     if dv is None:
-        dv = torch.empty_like(q)
+        dv = torch.empty_like(v)
     ws = int(layout._lib.st_attn_bwd_workspace_bytes(_c.byref(desc), layout.handle))
     if workspace is None:
         workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device)
@@ -198,15 +209,16 @@ def st_attn_bwd(q, k, v, o, lse, do, layout: Layout, dq=None, dk=None, dv=None, 
 
 def st_attn_decode(q, k_cache, v_cache, layout: Layout, pos: int, o=None, lse=None, workspace=None,
                    stream=None):
-    """Decode step: q [B, H, 64] at position pos against k_cache, v_cache [B, H, n, 64] (rows past
-    pos unread).  Returns o [B, H, 64] and lse [B, H] (fp32) -- row pos of the forward pass."""
-    _check_tensors(k_cache, v_cache)
+    """Decode step: q [B, H, d] at position pos against k_cache [B, H, n, d] and v_cache
+    [B, H, n, dv] (rows past pos unread; the kernels take d = dv = 64).  Returns o [B, H, dv] and
+    lse [B, H] (fp32) -- row pos of the forward pass."""
+    _check_tensors((k_cache,), (v_cache,))
     if not (q.is_cuda and q.is_contiguous() and q.dtype == k_cache.dtype and q.device == k_cache.device
             and q.dim() == 3 and tuple(q.shape) == (k_cache.shape[0], k_cache.shape[1], k_cache.shape[3])):
-        raise ValueError("q must be a contiguous [B, H, 64] CUDA tensor matching the caches")
-    desc = _desc(k_cache)
+        raise ValueError("q must be a contiguous [B, H, d] CUDA tensor matching the key cache")
+    desc = _desc(k_cache, v_cache)
     if o is None:
-        o = torch.empty_like(q)
+        o = q.new_empty((q.shape[0], q.shape[1], v_cache.shape[3]))
     if lse is None:
         lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
     ws = int(layout._lib.st_attn_decode_workspace_bytes(_c.byref(desc), layout.handle))

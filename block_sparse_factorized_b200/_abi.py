@@ -46,7 +46,7 @@ class st_pattern_t(ctypes.Structure):
 
 class st_desc_t(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("heads", ctypes.c_int64), ("n", ctypes.c_int64),
-                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("dv", ctypes.c_int32)]
 
 
 class st_layout_info_t(ctypes.Structure):

@@ -170,15 +170,22 @@ Frames frames_used(const st_layout &L)
     return f;
 }
 
+// Row widths the kernels are built for: query-key and value rows of 64 elements.
+bool widths_supported(const st_desc_t *desc)
+{
+    const int64_t dv = desc->dv == 0 ? desc->d : desc->dv;
+    return desc->d == 64 && dv == 64;
+}
+
 st_status_t check_common(const st_layout *L, const st_desc_t *desc)
 {
     if (!L || !desc) return ST_ERR_INVALID_ARG;
-    if (desc->reserved != 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
+    if (desc->dv < 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
         return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L->pat.num_heads || desc->n != L->n) return ST_ERR_INVALID_ARG;
     if (!L->exec_ok) return ST_ERR_UNSUPPORTED;
-    if (desc->d != 64) return ST_ERR_UNSUPPORTED;
+    if (!widths_supported(desc)) return ST_ERR_UNSUPPORTED;
     if (desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
     if (!L->uploaded) return ST_ERR_NOT_UPLOADED;
     int dev = -1;
@@ -486,11 +493,11 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
 {
     if (!q || !k_cache || !v_cache || !o || !lse || !layout || !desc) return ST_ERR_INVALID_ARG;
     const st_layout &L = *layout;
-    if (desc->reserved != 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
+    if (desc->dv < 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
         return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L.pat.num_heads || desc->n != L.n || pos < 0 || pos >= L.n) return ST_ERR_INVALID_ARG;
-    if (desc->d != 64 || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
+    if (!widths_supported(desc) || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
         return ST_ERR_ALIGNMENT;
     if (!workspace || workspace_bytes < st_attn_decode_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;

@@ -78,6 +78,13 @@ def test_argument_errors():
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 4
     d = _abi.st_desc_t(1, 2, 256, 32, 1, 0)
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 2
+    # value width: 0 or 64 pass the width check (NOT_UPLOADED next), other widths are valid but
+    # unsupported, a negative width is invalid
+    for dv, want in ((64, 4), (128, 2), (32, 2), (-1, 1)):
+        d = _abi.st_desc_t(1, 2, 256, 64, 1, dv)
+        assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == want
+        assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
+                               ctypes.byref(d), None) == want
     d = _abi.st_desc_t(1, 3, 256, 64, 1, 0)      # heads mismatch
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
     d = _abi.st_desc_t(1, 2, 256, 64, 7, 0)      # bad dtype
@@ -118,6 +125,8 @@ def test_decode_argument_errors():
     assert call(desc=_abi.st_desc_t(1, 3, 256, 64, 1, 0)) == 1   # heads are not the layout's
     assert call(desc=_abi.st_desc_t(1, 2, 512, 64, 1, 0)) == 1   # n is not the layout's
     assert call(desc=_abi.st_desc_t(1, 2, 256, 32, 1, 0)) == 2   # d != 64
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, 128)) == 2  # value width != 64
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, -1)) == 1   # negative value width
     assert call(q=odd) == 3                       # misaligned
     assert call(w=None) == 8 and call(wb=need - 1) == 8          # workspace missing / too small
     keys = np.empty(256, dtype=np.int64)
