@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "decode.h"
 #include "kernels.h"
 #include "layout.h"
@@ -32,18 +34,24 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode()
+{
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    return nullptr;
+}
+
+// The driver's tensor-map encoder, looked up once (thread-safe static initialisation; a failed
+// lookup is retried by the next call).
 EncodeTiledFn encode_fn()
 {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
+    static std::atomic<EncodeTiledFn> fn{lookup_encode()};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f && (f = lookup_encode())) fn.store(f, std::memory_order_release);
+    return f;
 }
 
 bool encode(CUtensorMap *m, const void *base, CUtensorMapDataType dt, cuuint32_t rank,
@@ -177,11 +185,19 @@ bool widths_supported(const st_desc_t *desc)
     return desc->d == 64 && dv == 64;
 }
 
+// Sizes every call and workspace query accepts: positive, and few enough rows (batch x heads x n
+// <= 2^40) that no byte count below can wrap.
+bool sizes_valid(const st_desc_t *desc)
+{
+    return desc->dv >= 0 && desc->batch >= 1 && desc->heads >= 1 && desc->n >= 1 && desc->d >= 1 &&
+           desc->batch <= (1ll << 30) && desc->heads <= (1ll << 30) && desc->n <= (1ll << 40) &&
+           desc->batch * desc->heads <= (1ll << 40) / desc->n;
+}
+
 st_status_t check_common(const st_layout *L, const st_desc_t *desc)
 {
     if (!L || !desc) return ST_ERR_INVALID_ARG;
-    if (desc->dv < 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
-        return ST_ERR_INVALID_ARG;
+    if (!sizes_valid(desc)) return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L->pat.num_heads || desc->n != L->n) return ST_ERR_INVALID_ARG;
     if (!L->exec_ok) return ST_ERR_UNSUPPORTED;
@@ -220,14 +236,14 @@ extern "C" {
 
 size_t st_attn_fwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    if (!desc || !layout) return 0;
+    if (!desc || !layout || !sizes_valid(desc)) return 0;
     // the unit counters of the two passes; fp32 I/O adds bf16 copies Q_hi, Q_lo, K_hi, K_lo, V_hi
     return FWD_SCHED_BYTES + (desc->dtype == ST_FP32 ? 5 * bf16_copy_bytes(desc) : 0);
 }
 
 size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    if (!desc || !layout) return 0;
+    if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
     const size_t dq = rows * 64 * sizeof(float);
     const size_t dl = rows * sizeof(float);
@@ -482,7 +498,7 @@ st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void 
 
 size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    if (!desc || !layout || desc->batch < 1 || desc->heads < 1 || desc->n < 1) return 0;
+    if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t nsplit = static_cast<size_t>((desc->n + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
     return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * st::DEC_PART * sizeof(float));
 }
@@ -493,8 +509,7 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
 {
     if (!q || !k_cache || !v_cache || !o || !lse || !layout || !desc) return ST_ERR_INVALID_ARG;
     const st_layout &L = *layout;
-    if (desc->dv < 0 || desc->batch < 1 || desc->heads < 1 || desc->n < 1 || desc->d < 1)
-        return ST_ERR_INVALID_ARG;
+    if (!sizes_valid(desc)) return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L.pat.num_heads || desc->n != L.n || pos < 0 || pos >= L.n) return ST_ERR_INVALID_ARG;
     if (!widths_supported(desc) || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;

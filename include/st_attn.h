@@ -172,7 +172,8 @@ ST_API st_status_t st_layout_check(st_layout_t *layout, st_stream_t stream);
 
 ST_API void st_layout_destroy(st_layout_t *layout);
 
-/* Workspace (device bytes, 256-byte aligned) the calls below need; 0 means none (NULL ok). */
+/* Workspace (device bytes, 256-byte aligned) the calls below need.  0 for a NULL argument or a
+ * descriptor whose sizes are invalid (non-positive, or batch x heads x n above 2^40 rows). */
 ST_API size_t st_attn_fwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout);
 ST_API size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *layout);
 

@@ -94,6 +94,14 @@ def test_argument_errors():
     assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
                            ctypes.byref(d), None) == 4
     assert lib.st_layout_check(lay.handle, None) == 4
+    # sizes that are not positive, or so many rows that byte counts could wrap, are invalid
+    # arguments; the workspace queries answer 0 for them
+    for bad in ((0, 2, 256, 64), (1, 2, 256, 0), (1 << 31, 2, 256, 64), (1 << 20, 2, 1 << 30, 64)):
+        d = _abi.st_desc_t(*bad, 1, 0)
+        assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
+        assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 0
+        assert lib.st_attn_bwd_workspace_bytes(ctypes.byref(d), lay.handle) == 0
+        assert lib.st_attn_decode_workspace_bytes(ctypes.byref(d), lay.handle) == 0
     # the forward always takes a workspace: the persistent kernel's unit counters come first
     d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
     assert lib.st_attn_fwd_workspace_bytes(ctypes.byref(d), lay.handle) == 256
