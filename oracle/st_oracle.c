@@ -351,17 +351,22 @@ void oracle_bwd_rows(const double *q, const double *k, const double *v, const do
     }
 }
 
-/* dK (nkeys x d) and dV (nkeys x e) for a chosen list of flat key rows r = (b*H + h)*n + j.  The
- * lse and D of every row of each (batch, head) that owns a chosen key are evaluated first (plain
- * row formulas). */
+/* dK (nkeys x d) and dV (nkeys x e) for a chosen list of flat key rows r = (b*H + h)*n + j.  Key j's
+ * gradients sum over the rows i that read it (j in A(i)), using those rows' lse and D; so the
+ * lse and D of exactly those rows are evaluated first (plain row formulas), found by the same
+ * predicate scan as bwd_key's. */
 void oracle_bwd_keys(const double *q, const double *k, const double *v, const double *dout,
                      int64_t B, int64_t H, int64_t n, int64_t d, int64_t e, const int *kind,
                      const int64_t *off, int64_t l, int64_t c, int64_t nkeys, const int64_t *keys,
                      double *dk_rows, double *dv_rows)
 {
     const int64_t nbh = B * H;
-    char *need = (char *)calloc((size_t)nbh, 1);
-    for (int64_t a = 0; a < nkeys; ++a) need[keys[a] / n] = 1;
+    char *need = (char *)calloc((size_t)(nbh * n), 1);
+    for (int64_t a = 0; a < nkeys; ++a) {
+        const int64_t r = keys[a], bh = r / n, j = r % n, h = bh % H;
+        for (int64_t i = j; i < n; ++i)
+            if (oracle_allowed(kind[h], i, j, l, c, off[h])) need[bh * n + i] = 1;
+    }
     double *lse = (double *)malloc(sizeof(double) * (size_t)(nbh * n));
     double *D = (double *)malloc(sizeof(double) * (size_t)(nbh * n));
 #pragma omp parallel
@@ -372,7 +377,7 @@ void oracle_bwd_keys(const double *q, const double *k, const double *v, const do
 #pragma omp for schedule(dynamic, 32)
         for (int64_t r = 0; r < nbh * n; ++r) {
             const int64_t bh = r / n, i = r % n, h = bh % H;
-            if (!need[bh]) continue;
+            if (!need[r]) continue;
             const size_t bq = (size_t)bh * (size_t)n * (size_t)d, bv = (size_t)bh * (size_t)n * (size_t)e;
             bwd_row(q + bq, k + bq, v + bv, dout + bv, d, e, kind[h], l, c, off[h], i, set, s, dp,
                     lse + r, D + r, NULL);
