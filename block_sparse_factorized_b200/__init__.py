@@ -162,6 +162,18 @@ def _ptr(t):
     return _c.c_void_p(t.data_ptr()) if t is not None else _c.c_void_p()
 
 
+def _workspace_bytes(workspace, device) -> int:
+    """Size in bytes of a caller's workspace tensor (any dtype), which must be a contiguous CUDA
+    tensor on the call's device; the C side checks it against the size the call needs."""
+    if workspace is None:
+        return 0
+    if not workspace.is_cuda or workspace.device != device:
+        raise ValueError("workspace must be a CUDA tensor on the inputs' device")
+    if not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    return workspace.numel() * workspace.element_size()
+
+
 def st_attn_fwd_workspace_bytes(q: torch.Tensor, layout: Layout) -> int:
     d = _desc(q)
     return int(layout._lib.st_attn_fwd_workspace_bytes(_c.byref(d), layout.handle))
@@ -172,8 +184,15 @@ def st_attn_bwd_workspace_bytes(q: torch.Tensor, layout: Layout) -> int:
     return int(layout._lib.st_attn_bwd_workspace_bytes(_c.byref(d), layout.handle))
 
 
-def st_attn_fwd(q, k, v, layout: Layout, o=None, lse=None, workspace=None, stream=None):
-    """O and lse ([B, H, n] fp32, natural log) of factorized sparse attention."""
+def st_attn_fwd(q, k, v, layout: Layout, o=None, lse=None, workspace=None, stream=None,
+                check=False):
+    """O and lse ([B, H, n] fp32, natural log) of factorized sparse attention.
+
+    The call is asynchronous.  A kernel whose bounded device wait ran out (a stalled pipeline,
+    e.g. on a heavily shared GPU) leaves O and lse partly written and records
+    ST_ERR_DEVICE_TIMEOUT in the layout's device error word: call ``layout.check()`` before
+    trusting the outputs, or pass ``check=True`` to have this call synchronise the stream and
+    raise StError on such an error."""
     _check_tensors((q, k), (v,) if o is None else (v, o))
     desc = _desc(q, v)
     B, H, n, _ = q.shape
@@ -185,15 +204,20 @@ def st_attn_fwd(q, k, v, layout: Layout, o=None, lse=None, workspace=None, strea
     if ws and workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
     st = layout._lib.st_attn_fwd(_ptr(q), _ptr(k), _ptr(v), layout.handle, _ptr(o), _ptr(lse),
-                                 _ptr(workspace), ws if workspace is not None else 0,
+                                 _ptr(workspace), _workspace_bytes(workspace, q.device),
                                  _c.byref(desc), _stream(stream))
     _abi.check(st, "st_attn_fwd")
+    if check:
+        layout.check(stream)
     return o, lse
 
 
 def st_attn_bwd(q, k, v, o, lse, do, layout: Layout, dq=None, dk=None, dv=None, workspace=None,
-                stream=None):
-    """dQ, dK, dV of factorized sparse attention (recomputing P from the saved lse)."""
+                stream=None, check=False):
+    """dQ, dK, dV of factorized sparse attention (recomputing P from the saved lse).
+
+    Asynchronous like st_attn_fwd: check the layout (``layout.check()``, or ``check=True`` here)
+    before trusting the gradients, since a device wait that ran out leaves them partly written."""
     _check_tensors((q, k), (v, o, do))
     desc = _desc(q, v)
     if dq is None:
@@ -207,8 +231,10 @@ def st_attn_bwd(q, k, v, o, lse, do, layout: Layout, dq=None, dk=None, dv=None, 
         workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device)
     st = layout._lib.st_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                  layout.handle, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-                                 workspace.numel(), _c.byref(desc), _stream(stream))
+                                 _workspace_bytes(workspace, q.device), _c.byref(desc), _stream(stream))
     _abi.check(st, "st_attn_bwd")
+    if check:
+        layout.check(stream)
     return dq, dk, dv
 
 
@@ -230,8 +256,8 @@ def st_attn_decode(q, k_cache, v_cache, layout: Layout, pos: int, o=None, lse=No
     if workspace is None:
         workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=q.device)
     st = layout._lib.st_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), layout.handle, int(pos), _ptr(o),
-                                    _ptr(lse), _ptr(workspace), workspace.numel(), _c.byref(desc),
-                                    _stream(stream))
+                                    _ptr(lse), _ptr(workspace), _workspace_bytes(workspace, q.device),
+                                    _c.byref(desc), _stream(stream))
     _abi.check(st, "st_attn_decode")
     return o, lse
 

@@ -12,6 +12,7 @@
 // contents; the prepare phase rewrites everything the main phase reads (the dQ accumulator is
 // zeroed, D recomputed), so no state leaks from one call to the next.  Two calls whose work
 // overlaps on the GPU (different streams, or another thread) race on the array.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -21,24 +22,56 @@
 namespace {
 
 // The scratch array itself.  In host code `scratch` names a host-side stand-in, not a device
-// address: the device address comes from cudaGetSymbolAddress, once per device.
+// address: the device address comes from cudaGetSymbolAddress, once per device and context.
 static __device__ __align__(256) unsigned char scratch[ST_NOALLOC_SCRATCH_BYTES];
 
 constexpr int MAX_DEVICES = 64;
 std::mutex scratch_mutex;
 void *scratch_ptr[MAX_DEVICES] = {};
+unsigned long long scratch_ctx[MAX_DEVICES] = {};  // context id the address belongs to
 
-// Device address of `scratch` on the current device; looked up on the first call per device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+template <typename F>
+F driver_fn(const char *name)
+{
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<F>(ptr);
+    return nullptr;
+}
+
+// Process-unique id of the current context (ids are never reused, unlike context handles), so
+// that an address looked up before a cudaDeviceReset is not reused in the context that follows.
+st_status_t current_context_id(unsigned long long *id)
+{
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return ST_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return ST_ERR_CUDA;
+    return get_id(ctx, id) == CUDA_SUCCESS ? ST_OK : ST_ERR_CUDA;
+}
+
+// Device address of `scratch` on the current device; looked up on the first call per device
+// (and again on the first call after that device's context was replaced).
 st_status_t scratch_address(void **out)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
     if (dev < 0 || dev >= MAX_DEVICES) return ST_ERR_UNSUPPORTED;
+    if (cudaSetDevice(dev) != cudaSuccess) return ST_ERR_CUDA;  // makes the device's primary context current
+    unsigned long long ctx = 0;
+    const st_status_t s = current_context_id(&ctx);
+    if (s != ST_OK) return s;
     std::lock_guard<std::mutex> lock(scratch_mutex);
-    if (!scratch_ptr[dev]) {
+    if (!scratch_ptr[dev] || scratch_ctx[dev] != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, scratch) != cudaSuccess || !p) return ST_ERR_CUDA;
         scratch_ptr[dev] = p;
+        scratch_ctx[dev] = ctx;
     }
     *out = scratch_ptr[dev];
     return ST_OK;

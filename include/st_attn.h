@@ -247,10 +247,15 @@ ST_API st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void 
  * the library's device image, held on every GPU that loads the library until the process exits.
  * Nothing is allocated (no cudaMalloc, cudaFree or allocating library call).
  *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
- *   - Problems whose st_attn_bwd_workspace_bytes exceeds ST_NOALLOC_SCRATCH_BYTES are rejected
- *     with ST_ERR_WORKSPACE before anything is enqueued (with bf16 I/O that is batch * heads * n
- *     above about 129,000 rows).
+ *     that device current); make that first call before any stream capture.  The address is
+ *     tied to the device's context: after a cudaDeviceReset the next call looks it up again
+ *     (that call too should come before any stream capture).
+ *   - The limit: a call is accepted when st_attn_bwd_workspace_bytes(desc, layout) <=
+ *     ST_NOALLOC_SCRATCH_BYTES; larger problems are rejected with ST_ERR_WORKSPACE before
+ *     anything is enqueued.  The workspace grows with batch * heads * n and also holds the
+ *     partial dK/dV of split key tiles and, for fp32 I/O, bf16 copies of the inputs, so the row
+ *     count alone is only an upper bound: with bf16 I/O and no split key tiles, batch * heads * n
+ *     up to about 129,000 rows.
  *   - All calls on a device share the array; each call re-initialises what it reads, but calls
  *     whose work overlaps on the GPU (other streams, other threads) race on it. */
 #define ST_NOALLOC_SCRATCH_BYTES (32u << 20)

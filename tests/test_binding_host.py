@@ -54,3 +54,36 @@ def test_descriptor_widths():
         bsf._desc(q.half())
     with pytest.raises(ValueError):
         bsf._desc(q[0])
+
+
+class FakeWorkspace(FakeCuda):
+    """A workspace tensor stand-in with a dtype of its own: the binding must send its real size."""
+
+    def __init__(self, numel, dtype, device="cuda:0", contiguous=True, is_cuda=True):
+        super().__init__((numel,), dtype, device)
+        self._n, self._contig, self.is_cuda = numel, contiguous, is_cuda
+
+    def numel(self):
+        return self._n
+
+    def element_size(self):
+        return torch.tensor([], dtype=self.dtype).element_size()
+
+    def is_contiguous(self):
+        return self._contig
+
+
+def test_workspace_size_is_the_buffer_size_in_bytes():
+    """The C side compares the byte count the binding sends with what the call needs, so the
+    binding sends the caller's buffer size (numel x element size), never the size the library
+    asked for."""
+    assert bsf._workspace_bytes(None, "cuda:0") == 0
+    assert bsf._workspace_bytes(FakeWorkspace(1000, torch.uint8), "cuda:0") == 1000
+    assert bsf._workspace_bytes(FakeWorkspace(1000, torch.float32), "cuda:0") == 4000
+    assert bsf._workspace_bytes(FakeWorkspace(10, torch.bfloat16), "cuda:0") == 20
+    with pytest.raises(ValueError):
+        bsf._workspace_bytes(FakeWorkspace(1000, torch.uint8, device="cuda:1"), "cuda:0")
+    with pytest.raises(ValueError):
+        bsf._workspace_bytes(FakeWorkspace(1000, torch.uint8, contiguous=False), "cuda:0")
+    with pytest.raises(ValueError):
+        bsf._workspace_bytes(torch.zeros(1000, dtype=torch.uint8), "cuda:0")  # a CPU tensor

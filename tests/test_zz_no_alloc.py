@@ -4,8 +4,9 @@ Such callers (a plug-in whose host application owns every device allocation, or 
 afford cudaMalloc's implicit synchronisation) get their scratch from a fixed array inside the
 library.  These tests call the entry point through the C ABI and check that two calls in a row
 give the same gradients as the ordinary st_attn_bwd with a caller-provided workspace, within the
-gradient tolerance the other tests use, and that a problem too large for the fixed array is
-refused before anything runs.  The file is collected last on purpose.
+gradient tolerance the other tests use, that both calls also meet that tolerance against the fp64
+oracle, and that a problem too large for the fixed array is refused before anything runs.  The
+file is collected last on purpose.
 """
 import ctypes
 
@@ -13,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import GRAD_REL_L2, cuda_inputs, rel_l2, to64
+from parity import GRAD_REL_L2, check_grads, cuda_inputs, problem_of, rel_l2, to64
 from workloads import ALTERNATING, FIXED, MERGED, STRIDED, WORKLOADS, Workload
 
 pytestmark = pytest.mark.gpu
@@ -35,7 +36,8 @@ def _p(t):
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_noalloc_matches_workspace_entry_point_twice(w):
     lib = _abi.load()
-    (q, k, v, do), _ = cuda_inputs(w)
+    (q, k, v, do), host = cuda_inputs(w)
+    oracle_grads = problem_of(w).bwd(*(to64(t) for t in host))
     lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).upload()
     o, lse = bsf.st_attn_fwd(q, k, v, lay)
     ref = bsf.st_attn_bwd(q, k, v, o, lse, do, lay)
@@ -53,6 +55,7 @@ def test_noalloc_matches_workspace_entry_point_twice(w):
             assert torch.isfinite(got).all(), (call, name)
             err = rel_l2(to64(got), to64(want))
             assert err <= GRAD_REL_L2, (call, name, err)
+        check_grads((to64(dq), to64(dk), to64(dv)), oracle_grads, f"{w.name} call {call}")
 
 
 def test_noalloc_refuses_problems_beyond_the_fixed_scratch():
