@@ -1,8 +1,9 @@
 """Backward parity of the CUDA path (recomputing backward, through the C ABI binding) against the
 fp64 oracle's plain-calculus gradients.
 
-Small cases compare every element of dQ, dK and dV; the full-size workloads compare dQ on sampled
-query rows and dK, dV on sampled keys, each evaluated one by one by the oracle.  Keys that no
+Small cases compare every element of dQ, dK and dV; the long sequences (2^18 and 2^20 keys)
+compare dQ on sampled query rows and dK, dV on sampled keys, each evaluated one by one by the
+oracle (the benchmark workloads are compared on every element in test_full_size_gpu.py).  Keys that no
 query reads must get exactly zero gradient, rows with no allowed key exactly zero dQ.
 """
 import numpy as np
@@ -47,15 +48,12 @@ def test_bwd_small_all_elements(w):
         assert torch.all(dk[:, h, unread] == 0) and torch.all(dv[:, h, unread] == 0)
 
 
-BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
-# longer sequences (l about sqrt(n)), sampled rows: frames and work lists at 2^18 and 2^20 keys
-BIG += [Workload("s_n262144_l512_long", STRIDED, ALTERNATING, 262144, 512, 0, 1, 4),
-        Workload("s_merged_n262144_l512_long", STRIDED, MERGED, 262144, 512, 0, 1, 2),
-        Workload("s_n1048576_l1024_long", STRIDED, ALTERNATING, 1048576, 1024, 0, 1, 2),
-        Workload("f_n262144_l512_c128_long", FIXED, ALTERNATING, 262144, 512, 128, 1, 2)]
-# (the oracle's key-side gradients of a fixed-pattern summary key scan every later row and its
-# whole set: out of reach at 2^18 keys, so that case is checked in the forward only)
-BIG = [w for w in BIG if not w.name.startswith("f_n262144")]
+# longer sequences (l about sqrt(n)), sampled rows and keys: frames and work lists at 2^18 and 2^20
+# keys (the benchmark workloads are compared on every element in test_full_size_gpu.py)
+BIG = [Workload("s_n262144_l512_long", STRIDED, ALTERNATING, 262144, 512, 0, 1, 4),
+       Workload("s_merged_n262144_l512_long", STRIDED, MERGED, 262144, 512, 0, 1, 2),
+       Workload("s_n1048576_l1024_long", STRIDED, ALTERNATING, 1048576, 1024, 0, 1, 2),
+       Workload("f_n262144_l512_c128_long", FIXED, ALTERNATING, 262144, 512, 128, 1, 2)]
 
 
 @pytest.mark.parametrize("w", FP32, ids=lambda w: w.name)
@@ -68,16 +66,25 @@ def test_bwd_fp32_all_elements(w):
 
 
 def sample_keys(w, count, seed=1):
+    """Flat key indices (b*H + h)*n + j: block and tile edges of every head plus random keys.  A
+    summary key of the fixed pattern's second head (or of a merged fixed head) is read by every
+    later row, and the oracle evaluates each reading row in full; at 2^18 keys those heads are
+    sampled in their last two blocks only, where the reading rows are few.  Same-block and strided
+    heads are sampled anywhere."""
     rng = np.random.default_rng(seed)
+    kinds, _ = oracle.head_kinds(w.family, w.head_mode, w.heads, w.l, w.c, w.offset_step)
     keys = set()
     for b in range(w.batch):
         for h in range(w.heads):
             base = (b * w.heads + h) * w.n
-            for j in (0, w.l - 1, w.l - w.c - 1 if w.c else 1, 127, 128, w.n // 2 - 1, w.n - 1):
-                if 0 <= j < w.n:
+            late = w.n >= (1 << 18) and int(kinds[h]) in (oracle.FA2, oracle.FU)
+            lo = w.n - 2 * w.l if late else 0
+            edges = (0, w.l - 1, w.l - w.c - 1 if w.c else 1, 127, 128, w.n // 2 - 1, w.n - 1)
+            for j in edges:
+                if lo <= j < w.n:
                     keys.add(base + j)
-    total = w.batch * w.heads * w.n
-    keys.update(rng.integers(0, total, size=count).tolist())
+            per_head = max(1, count // (w.batch * w.heads))
+            keys.update((base + rng.integers(lo, w.n, size=per_head)).tolist())
     return np.array(sorted(keys), dtype=np.int64)
 
 
@@ -161,3 +168,22 @@ def test_bwd_phases_and_direct_dq(w):
             assert rel_l2(to64(dq1[:, h]), to64(dq2[:, h])) < 1e-3, h
     ref = problem_of(w).bwd(to64(q), to64(k), to64(v), to64(do))
     check_grads((to64(dq2), to64(dk2), to64(dv2)), ref, w.name)
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[7], SMALL[15]], ids=lambda w: w.name)
+def test_bwd_guard_zones(w):
+    """dQ, dK and dV written into views with guard zones on both sides: the backward pass (TMA
+    stores clipped at the frame edges, the dK/dV partials of split key tiles, merge passes) writes
+    nothing outside its outputs, and the gradients still match the oracle."""
+    (qd, kd, vd, dod), (q, k, v, do) = cuda_inputs(w)
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).upload()
+    o, lse = bsf.st_attn_fwd(qd, kd, vd, lay)
+    numel, guard = qd.numel(), 8192
+    bufs = [torch.full((numel + 2 * guard,), 7.0, dtype=qd.dtype, device=qd.device) for _ in range(3)]
+    dq, dk, dv = (b[guard:guard + numel].view_as(qd) for b in bufs)
+    bsf.st_attn_bwd(qd, kd, vd, o, lse, dod, lay, dq=dq, dk=dk, dv=dv, check=True)
+    torch.cuda.synchronize()
+    for b in bufs:
+        assert torch.all(b[:guard] == 7.0) and torch.all(b[-guard:] == 7.0)
+    ref = problem_of(w).bwd(to64(q), to64(k), to64(v), to64(do))
+    check_grads((to64(dq), to64(dk), to64(dv)), ref, w.name)

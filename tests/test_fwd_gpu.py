@@ -1,7 +1,8 @@
 """Forward parity of the CUDA path (through the C ABI binding) against the fp64 oracle.
 
-Small cases compare every element; the full-size workloads compare sampled rows evaluated one by
-one by the oracle, in the same launch configuration the benchmark times.  Invariants that hold at
+Small cases compare every element; the long sequences (2^18 and 2^20 keys) compare sampled rows
+evaluated one by one by the oracle (the benchmark workloads are compared on every element in
+test_full_size_gpu.py).  Invariants that hold at
 any size (Q = 0 closed form, masked-V perturbation, determinism, guard zones) run on the GPU too.
 """
 import math
@@ -64,9 +65,9 @@ def test_fwd_small_all_elements(w):
     check_o_lse(to64(o), lse.cpu().numpy(), o_ref, lse_ref, w.name)
 
 
-BIG = [w for w in WORKLOADS.values() if w.dtype == "bf16"]
 # longer sequences (l about sqrt(n)), sampled rows: frames and work lists at 2^18 and 2^20 keys
-BIG += [Workload("s_n262144_l512_long", STRIDED, ALTERNATING, 262144, 512, 0, 1, 4),
+# (the benchmark workloads themselves are compared on every element in test_full_size_gpu.py)
+BIG = [Workload("s_n262144_l512_long", STRIDED, ALTERNATING, 262144, 512, 0, 1, 4),
         Workload("s_merged_n262144_l512_long", STRIDED, MERGED, 262144, 512, 0, 1, 2),
         Workload("s_n1048576_l1024_long", STRIDED, ALTERNATING, 1048576, 1024, 0, 1, 2),
         Workload("f_n262144_l512_c128_long", FIXED, ALTERNATING, 262144, 512, 128, 1, 2)]
@@ -181,3 +182,21 @@ def test_fwd_deterministic_and_guarded():
     assert torch.all(obuf[:guard] == 7.0) and torch.all(obuf[-guard:] == 7.0)
     assert torch.all(lbuf[:guard] == 7.0) and torch.all(lbuf[-guard:] == 7.0)
     lay.check()
+
+
+def test_fwd_workspace_too_small_is_refused():
+    """A caller's workspace smaller than st_attn_fwd_workspace_bytes is refused with
+    ST_ERR_WORKSPACE before anything runs, whatever the workspace tensor's dtype (the binding
+    sends its size in bytes)."""
+    w = FP32[1]  # fp32 I/O: the forward's workspace holds the bf16 high/low copies of q, k, v
+    (qd, kd, vd, _), _ = cuda_inputs(w)
+    lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).upload()
+    need = bsf.st_attn_fwd_workspace_bytes(qd, lay)
+    assert need > 1 << 16
+    small = torch.empty(need // 8, dtype=torch.float32, device=qd.device)  # need / 2 bytes
+    with pytest.raises(bsf.StError) as e:
+        bsf.st_attn_fwd(qd, kd, vd, lay, workspace=small)
+    assert e.value.status == 8  # ST_ERR_WORKSPACE
+    ok = torch.empty(need // 4 + 1, dtype=torch.float32, device=qd.device)
+    o, lse = bsf.st_attn_fwd(qd, kd, vd, lay, workspace=ok, check=True)
+    assert torch.isfinite(o).all()

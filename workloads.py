@@ -7,9 +7,10 @@ Recipe: one CPU ``torch.Generator`` seeded with ``seed`` (0 by default) draws Q,
 that order, as iid N(0, 1) fp32 of shape [batch, heads, n, d]; each is then rounded to the
 workload's I/O dtype.  The oracle gets those rounded values widened to fp64.
 
-The five workloads stand in for the pages' data (no dataset is needed or present): a 32x32x3
-image raster (n = 3072), Enwik8-length text (n = 12288, l = 128, c = 32), a 64x64x3 raster
-(n = 12288, stride 128) and a 65,536-sample audio clip (l = 256), plus a small fp32 case.
+The workloads stand in for the pages' data (no dataset is needed or present): a 32x32x3 image
+raster (n = 3072), Enwik8-length text (n = 12288, l = 128, c = 32; per-head alternating, and
+merged heads as the text model uses them), a 64x64x3 raster (n = 12288, stride 128) and a
+65,536-sample audio clip (l = 256), plus a small fp32 case.
 """
 from __future__ import annotations
 
@@ -60,6 +61,10 @@ WORKLOADS = {
                                            128, 0, 2, 16),
     "strided_n65536_l256": Workload("strided_n65536_l256", STRIDED, ALTERNATING, 65536, 256, 0,
                                     1, 8),
+    # the text model's own setting: fixed pattern with merged heads (each head reads its block and
+    # every earlier block's summary run), n = 12288, l = 128, c = 32, 8 heads
+    "fixed_merged_n12288_l128_c32": Workload("fixed_merged_n12288_l128_c32", FIXED, MERGED, 12288,
+                                             128, 32, 2, 8),
 }
 
 # The headline workload: fixed pattern, text-shaped, n = 12288.
