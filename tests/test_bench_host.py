@@ -58,6 +58,29 @@ def test_reference_arm_json_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
 
 
+def test_reference_arm_loads_no_cuda_library():
+    """The reference arm is the oracle alone: running it maps liboracle.so but never the CUDA
+    library (its FLOP count comes from the canonical tile table)."""
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', "
+            "'--warmup', '0', '--workload', 'strided_n256_l16_fp32']\n"
+            "try:\n    runpy.run_path('bench.py', run_name='__main__')\nexcept SystemExit:\n    pass\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "print('LIBST' if 'libst_attn' in maps else 'NOLIBST', 'ORACLE' if 'liboracle' in maps else 'NOORACLE')")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip().splitlines()[-1] == "NOLIBST ORACLE"
+
+
+def test_canonical_tile_table_matches_the_library_census():
+    import block_sparse_factorized_b200 as bsf
+    from workloads import WORKLOADS
+    assert set(bench.CANONICAL_TILES) == set(WORKLOADS)
+    for name, w in WORKLOADS.items():
+        info = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c).info()
+        assert bench.CANONICAL_TILES[name] == info["exec_tiles"], name
+        assert bench.canonical_flops(w) == bench.step_flops(w, info)[0], name
+
+
 def test_reference_arm_nonzero_ranks_exit_quietly():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
