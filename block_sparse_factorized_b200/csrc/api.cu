@@ -513,7 +513,8 @@ size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *
 {
     if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t nsplit = static_cast<size_t>((desc->n + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
-    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * st::DEC_PART * sizeof(float));
+    const size_t part = static_cast<size_t>(value_width(desc)) + 4;  // dec_part(dv) floats per chunk
+    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * part * sizeof(float));
 }
 
 st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache, const st_layout_t *layout,
@@ -525,7 +526,10 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     if (!sizes_valid(desc)) return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L.pat.num_heads || desc->n != L.n || pos < 0 || pos >= L.n) return ST_ERR_INVALID_ARG;
-    if (!widths_supported(desc) || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
+    const int64_t dv = value_width(desc);
+    if (desc->d > 128 || dv > 128 || !st::decode_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv)) ||
+        desc->heads > 64 || desc->batch * desc->heads > (1ll << 30))
+        return ST_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
         return ST_ERR_ALIGNMENT;
     if (!workspace || workspace_bytes < st_attn_decode_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
@@ -551,10 +555,11 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     p.c = L.c;
     p.bh = static_cast<int32_t>(desc->batch * desc->heads);
     p.heads = static_cast<int32_t>(desc->heads);
-    p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
+    p.scale_log2 = LOG2E / sqrtf(static_cast<float>(desc->d));  // log2(e) / sqrt(d)
     const int64_t nsplit = (most + st::DEC_CHUNK - 1) / st::DEC_CHUNK;
     if (nsplit > 65535) return ST_ERR_UNSUPPORTED;  // grid dimension y: a row with over 4 M allowed keys
-    return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, stream) == cudaSuccess
+    return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, static_cast<int>(desc->d),
+                             static_cast<int>(dv), stream) == cudaSuccess
                ? ST_OK
                : ST_ERR_CUDA;
 }

@@ -136,9 +136,13 @@ def test_decode_argument_errors():
     assert call(pos=-1) == 1 and call(pos=256) == 1   # position outside [0, n)
     assert call(desc=_abi.st_desc_t(1, 3, 256, 64, 1, 0)) == 1   # heads are not the layout's
     assert call(desc=_abi.st_desc_t(1, 2, 512, 64, 1, 0)) == 1   # n is not the layout's
-    assert call(desc=_abi.st_desc_t(1, 2, 256, 32, 1, 0)) == 2   # d != 64
-    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, 128)) == 2  # value width != 64
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, 32)) == 2   # no kernel for (64, 32)
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 48, 1, 0)) == 2    # nor for 48-wide rows
     assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, -1)) == 1   # negative value width
+    # the chunk record is dv + 4 floats: 2 x 4 x 132 x 4 bytes at dv = 128
+    wide = _abi.st_desc_t(1, 2, 256, 64, 1, 128)
+    assert lib.st_attn_decode_workspace_bytes(ctypes.byref(wide), lay.handle) == 4352
+    assert call(desc=wide) == 8                                  # the 64-wide workspace is too small
     assert call(q=odd) == 3                       # misaligned
     assert call(w=None) == 8 and call(wb=need - 1) == 8          # workspace missing / too small
     keys = np.empty(256, dtype=np.int64)
