@@ -8,6 +8,7 @@ encoder is looked up through the runtime's driver entry point, so no -lcuda is n
 """
 from __future__ import annotations
 
+import fcntl
 import glob
 import os
 import subprocess
@@ -38,10 +39,21 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile and link the library when it is missing or stale (always with force).  Builds by
+    several processes at once (test workers) are serialised by a lock on the object directory; a
+    process that waited re-checks staleness, so the library is built once."""
     if not force and not _stale():
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
+    with open(os.path.join(objdir, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        if not force and not _stale():
+            return LIB
+        return _compile_and_link(objdir, verbose)
+
+
+def _compile_and_link(objdir: str, verbose: bool) -> str:
     objs = []
     procs = []
     for src in sources():
