@@ -191,11 +191,12 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------- oracle sample (CPU)
-def oracle_sample(w, slabs):
+def oracle_sample(w, slabs, inputs=None):
     """Run the oracle's full forward + backward on the given (batch, head) slabs; return
-    (seconds, threads).  Each slab is one (b, h): the oracle runs the whole n for that head."""
+    (seconds, threads).  Each slab is one (b, h): the oracle runs the whole n for that head.
+    inputs: the workload's (q, k, v, do), drawn here when not given (outside the timing)."""
     import oracle
-    q, k, v, do = make_inputs(w)
+    q, k, v, do = inputs if inputs is not None else make_inputs(w)
     kinds, offs = oracle.head_kinds(w.family, w.head_mode, w.heads, w.l, w.c, w.offset_step)
     t0 = time.perf_counter()
     for b, h in slabs:
@@ -204,6 +205,27 @@ def oracle_sample(w, slabs):
         p.fwd(*sl[:3])
         p.bwd(*sl)
     return time.perf_counter() - t0, oracle.num_threads()
+
+
+CPU_BASELINE_SECONDS = 10.0  # oracle time per CPU-baseline measurement
+
+
+def cpu_baseline(w, flops, min_seconds=CPU_BASELINE_SECONDS):
+    """The oracle, as it stands, on the host cores: the full forward + backward of one (batch,
+    head) slab after another, cycling over the workload's slabs until at least min_seconds of
+    oracle time have run (at most 64 passes over the workload).  value = the metric's FLOPs per
+    workload x the workloads covered / the oracle time."""
+    inputs = make_inputs(w)
+    slabs = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    done, secs, threads = 0, 0.0, 1
+    while secs < min_seconds and done < 64 * len(slabs):
+        s, threads = oracle_sample(w, [slabs[done % len(slabs)]], inputs)
+        secs += s
+        done += 1
+    covered = done / len(slabs)
+    return {"value": flops * covered / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"oracle fwd+bwd of {done} (batch, head) slabs at full n={w.n}, cycling over the "
+                      f"workload's {len(slabs)} ({covered:.2f} workloads), {secs:.1f} s"}
 
 
 def step_flops(w, info):
@@ -244,9 +266,10 @@ def run_reference(args, rank, world):
     slabs_all = [(b, h) for b in range(w.batch) for h in range(w.heads)]
     per_step = []
     threads = 1
+    inputs = make_inputs(w)
     for s in range(args.warmup + args.steps):
         slab = slabs_all[s % len(slabs_all)] if w.head_mode == 2 else (0, s % w.heads)
-        secs, threads = oracle_sample(w, [slab])
+        secs, threads = oracle_sample(w, [slab], inputs)
         if s >= args.warmup:
             per_step.append(secs * len(slabs_all))   # time the whole workload would take
     ms = 1e3 * statistics.mean(per_step)
@@ -389,13 +412,7 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        slabs = [(0, h) for h in range(min(2, w.heads))]
-        secs, threads = oracle_sample(w, slabs)
-        scale = (w.batch * w.heads) / len(slabs)
-        cpu_val = flops / (secs * scale) / 1e12
-        cpu = {"value": cpu_val, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"oracle fwd+bwd of batch 0, heads 0-{len(slabs) - 1} (full n={w.n}), "
-                         f"{secs:.1f} s, scaled by {scale:g} to the whole workload"}
+        cpu = cpu_baseline(w, flops)
 
     clocks = sampler.summary()
     line = {

@@ -19,13 +19,13 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import (ST_BF16, ST_FIXED, ST_FP32, ST_KIND_FA1, ST_KIND_FA2, ST_KIND_FU, ST_KIND_SA1,
+from ._abi import (ST_BF16, ST_ERR_DEVICE_TIMEOUT, ST_FIXED, ST_FP32, ST_KIND_FA1, ST_KIND_FA2, ST_KIND_FU, ST_KIND_SA1,
                    ST_KIND_SA2, ST_KIND_SU, ST_MERGED, ST_PER_HEAD_ALTERNATING, ST_SINGLE_A1,
                    ST_SINGLE_A2, ST_STRIDED, StError)
 
 __all__ = [
     "Layout", "st_attn_fwd", "st_attn_bwd", "st_attn_decode", "st_attn_fwd_workspace_bytes",
-    "st_attn_bwd_workspace_bytes", "SparseAttention", "StError", "ST_STRIDED", "ST_FIXED",
+    "st_attn_bwd_workspace_bytes", "SparseAttention", "StError", "ST_ERR_DEVICE_TIMEOUT", "ST_STRIDED", "ST_FIXED",
     "ST_PER_HEAD_ALTERNATING", "ST_MERGED", "ST_SINGLE_A1", "ST_SINGLE_A2", "ST_BF16", "ST_FP32",
     "ST_KIND_SA1", "ST_KIND_SA2", "ST_KIND_SU", "ST_KIND_FA1", "ST_KIND_FA2", "ST_KIND_FU",
 ]
@@ -110,6 +110,11 @@ class Layout:
 
     def check(self, stream=None) -> None:
         _abi.check(self._lib.st_layout_check(self._h, _stream(stream)), "st_layout_check")
+
+    def selftest_wait_timeout(self, stream=None) -> None:
+        """Launch one warp whose bounded wait runs out (after 1 s): the next check() raises
+        StError with ST_ERR_DEVICE_TIMEOUT, and the context stays usable."""
+        _abi.check(self._lib.st_selftest_wait_timeout(self._h, _stream(stream)), "st_selftest_wait_timeout")
 
     def __del__(self):
         h = getattr(self, "_h", None)

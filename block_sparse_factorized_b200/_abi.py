@@ -12,6 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libst_attn.so")
 
 ST_OK = 0
+ST_ERR_DEVICE_TIMEOUT = 7
 STATUS_NAMES = {
     0: "ST_OK", 1: "ST_ERR_INVALID_ARG", 2: "ST_ERR_UNSUPPORTED", 3: "ST_ERR_ALIGNMENT",
     4: "ST_ERR_NOT_UPLOADED", 5: "ST_ERR_CUDA", 6: "ST_ERR_OOM", 7: "ST_ERR_DEVICE_TIMEOUT",
@@ -25,7 +26,8 @@ ST_KIND_SA1, ST_KIND_SA2, ST_KIND_SU, ST_KIND_FA1, ST_KIND_FA2, ST_KIND_FU = 1, 
 # every symbol include/st_attn.h declares
 EXPORTED = (
     "st_layout_build", "st_layout_upload", "st_layout_head_kind", "st_layout_export",
-    "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_layout_destroy",
+    "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_selftest_wait_timeout",
+    "st_layout_destroy",
     "st_attn_fwd_workspace_bytes", "st_attn_bwd_workspace_bytes", "st_attn_fwd", "st_attn_bwd",
     "st_attn_bwd_prepare", "st_attn_bwd_main", "st_attn_bwd_finish", "st_attn_bwd_noalloc",
     "st_attn_decode_workspace_bytes", "st_attn_decode", "st_decode_row_keys",
@@ -80,6 +82,7 @@ def load() -> ctypes.CDLL:
     lib.st_layout_info.argtypes = [P, pp(st_layout_info_t)]
     lib.st_layout_exec_row.argtypes = [P, i32, i64, P, pp(i64)]
     lib.st_layout_check.argtypes = [P, P]
+    lib.st_selftest_wait_timeout.argtypes = [P, P]
     lib.st_layout_destroy.argtypes = [P]
     lib.st_layout_destroy.restype = None
     lib.st_attn_fwd_workspace_bytes.argtypes = [pp(st_desc_t), P]
@@ -101,7 +104,8 @@ def load() -> ctypes.CDLL:
     lib.st_status_string.restype = ctypes.c_char_p
     lib.st_version.restype = ctypes.c_char_p
     for name in ("st_layout_build", "st_layout_upload", "st_layout_head_kind", "st_layout_export",
-                 "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_attn_fwd",
+                 "st_layout_info", "st_layout_exec_row", "st_layout_check", "st_selftest_wait_timeout",
+                 "st_attn_fwd",
                  "st_attn_bwd", "st_attn_bwd_prepare", "st_attn_bwd_main", "st_attn_bwd_finish",
                  "st_attn_decode", "st_decode_row_keys"):
         getattr(lib, name).restype = i32

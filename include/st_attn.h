@@ -22,8 +22,9 @@
  * bf16 split precision (error about 2^-16) and the rest in bf16 products, fp32 accumulation.
  *
  * Conventions for every call:
- *   - Tensors are contiguous row-major [batch, heads, n, d] (lse and the like [batch, heads, n]),
- *     in device memory owned by the caller, each 16-byte aligned.  d must be 64.
+ *   - Tensors are contiguous row-major [batch, heads, n, width] (lse and the like
+ *     [batch, heads, n]), in device memory owned by the caller, each 16-byte aligned; the row
+ *     widths are the descriptor's d (Q, K) and dv (V, O), both 64 for the kernels.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream) and
  *     return after enqueueing work; argument errors are reported before anything is enqueued.
  *   - No call allocates device memory except st_layout_upload (the layout's own tables).
@@ -170,6 +171,15 @@ ST_API st_status_t st_layout_exec_row(const st_layout_t *layout, int32_t head, i
 /* Synchronise `stream` and report (and clear) the layout's device error word:
  * ST_ERR_DEVICE_TIMEOUT if a kernel's bounded wait gave up since the last check. */
 ST_API st_status_t st_layout_check(st_layout_t *layout, st_stream_t stream);
+
+/* Diagnostic of the failure path: launches one warp on `stream` whose single bounded wait is on
+ * an mbarrier that nothing completes, so it gives up after the kernels' wait limit (1 s) and
+ * records the timeout in the layout's device error word, as a stalled kernel pipeline would.
+ * The next st_layout_check then returns ST_ERR_DEVICE_TIMEOUT (and clears the word); the CUDA
+ * context stays usable.  Lets a caller test its error handling without a real fault.
+ * Errors: ST_ERR_INVALID_ARG (NULL layout, or the current device is not the layout's),
+ * ST_ERR_NOT_UPLOADED, ST_ERR_CUDA (launch failed). */
+ST_API st_status_t st_selftest_wait_timeout(st_layout_t *layout, st_stream_t stream);
 
 ST_API void st_layout_destroy(st_layout_t *layout);
 

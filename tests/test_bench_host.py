@@ -86,3 +86,15 @@ def test_headline_flop_and_byte_counts():
     used = 2 * (4 * 12288 + 4 * 96 * 32)  # K/V rows read: 4 full heads + 4 summary heads
     assert fwd_b == 2 * rows * row + 2 * used * row + rows * 4
     assert bwd_b == fwd_b + rows * row + rows * 4 + 3 * rows * row
+
+
+def test_cpu_baseline_covers_whole_slabs():
+    """The CPU baseline runs the oracle on whole (batch, head) slabs, cycling over the workload
+    until the time floor is met, and reports throughput over the slabs it covered."""
+    from workloads import Workload, STRIDED, ALTERNATING
+    w = Workload("s_n512_l16", STRIDED, ALTERNATING, 512, 16, 0, 1, 2)
+    cpu = bench.cpu_baseline(w, flops=1e9, min_seconds=0.2)
+    assert cpu["kind"] == "oracle" and cpu["unit"] == "TFLOP/s" and cpu["cores"] >= 1
+    assert cpu["value"] > 0 and "slabs at full n=512" in cpu["sample"]
+    done = int(cpu["sample"].split("oracle fwd+bwd of ")[1].split()[0])
+    assert done >= 1

@@ -98,6 +98,8 @@ def test_argument_errors():
     assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
                            ctypes.byref(d), None) == 4
     assert lib.st_layout_check(lay.handle, None) == 4
+    assert lib.st_selftest_wait_timeout(None, None) == 1
+    assert lib.st_selftest_wait_timeout(lay.handle, None) == 4
     # sizes that are not positive, or so many rows that byte counts could wrap, are invalid
     # arguments; the workspace queries answer 0 for them
     for bad in ((0, 2, 256, 64), (1, 2, 256, 0), (1 << 31, 2, 256, 64), (1 << 20, 2, 1 << 30, 64)):
