@@ -129,7 +129,8 @@ ST_API st_status_t st_layout_build(const st_pattern_t *pattern, int64_t n, int32
  * run this layout (n % 128, n % l, c, heads > 64), ST_ERR_CUDA, ST_ERR_OOM. */
 ST_API st_status_t st_layout_upload(st_layout_t *layout, st_stream_t stream);
 
-/* Kind (st_kind_t) and fixed sub-block offset o of head `head`. */
+/* Kind (st_kind_t) and fixed sub-block offset o of head `head` (host only).
+ * Errors: ST_ERR_INVALID_ARG (NULL layout, head outside [0, num_heads)). */
 ST_API st_status_t st_layout_head_kind(const st_layout_t *layout, int32_t head, int32_t *kind,
                                 int32_t *offset);
 
@@ -147,7 +148,8 @@ ST_API st_status_t st_layout_export(const st_layout_t *layout, int32_t head, con
                              const uint32_t **masks, int32_t *n_qblk, int32_t *nnz,
                              int32_t *n_masks);
 
-/* Per batch element figures of the execution plan. */
+/* Per batch element figures of the execution plan (host only).  Errors: ST_ERR_INVALID_ARG
+ * (NULL argument), ST_ERR_UNSUPPORTED (a layout the kernels cannot run has no plan). */
 typedef struct {
     int64_t fwd_items;      /* forward work items (query tiles over all heads and passes) */
     int64_t exec_tiles;     /* active 128 x 128 tile pairs the kernels compute */
@@ -164,7 +166,9 @@ ST_API st_status_t st_layout_info(const st_layout_t *layout, st_layout_info_t *i
 
 /* Host enumeration of the keys row i of head `head` attends in the execution frames (the same
  * frame and interval rules the kernels use), increasing, written to keys[0 .. *count-1];
- * keys must hold n entries.  For tests of the execution plan against the set definitions. */
+ * keys must hold n entries.  For tests of the execution plan against the set definitions.
+ * Errors: ST_ERR_INVALID_ARG (NULL pointer, head or i out of range), ST_ERR_UNSUPPORTED (a
+ * layout the kernels cannot run has no plan). */
 ST_API st_status_t st_layout_exec_row(const st_layout_t *layout, int32_t head, int64_t i, int64_t *keys,
                                int64_t *count);
 
@@ -181,6 +185,8 @@ ST_API st_status_t st_layout_check(st_layout_t *layout, st_stream_t stream);
  * ST_ERR_NOT_UPLOADED, ST_ERR_CUDA (launch failed). */
 ST_API st_status_t st_selftest_wait_timeout(st_layout_t *layout, st_stream_t stream);
 
+/* Release the layout's host tables and device buffers (NULL is a no-op).  Work already enqueued
+ * that uses the layout must have completed. */
 ST_API void st_layout_destroy(st_layout_t *layout);
 
 /* Workspace (device bytes, 256-byte aligned) the calls below need.  0 for a NULL argument or a
@@ -193,7 +199,11 @@ ST_API size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout
  * second pass merges by log-sum-exp into the first pass's O and lse).
  * The workspace (st_attn_fwd_workspace_bytes, never 0) starts with the work-unit counters of the
  * persistent kernel, zeroed on `stream` by every call: calls that run at the same time need
- * separate workspaces.  fp32 I/O adds the bf16 copies of q, k and v after them. */
+ * separate workspaces.  fp32 I/O adds the bf16 copies of q, k and v after them.
+ * Errors (nothing enqueued): ST_ERR_INVALID_ARG (NULL pointer; descriptor sizes, heads or n not
+ * the layout's; the current device is not the layout's), ST_ERR_UNSUPPORTED (row widths or a
+ * layout the kernels do not handle), ST_ERR_ALIGNMENT, ST_ERR_NOT_UPLOADED, ST_ERR_WORKSPACE;
+ * ST_ERR_CUDA if a launch fails. */
 ST_API st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_layout_t *layout,
                         void *o, float *lse, void *workspace, size_t workspace_bytes,
                         const st_desc_t *desc, st_stream_t stream);
@@ -201,7 +211,8 @@ ST_API st_status_t st_attn_fwd(const void *q, const void *k, const void *v, cons
 /* Backward pass with recomputation ("Sparse Transformers 深度解读报告" §3.4): attention
  * probabilities are rebuilt from q, k and the saved lse.  o, dO: forward output and its
  * gradient; dq, dk, dv: outputs (every element written; keys no query reads get 0).
- * The workspace holds the fp32 dQ accumulator and the per-row D_i = dO_i . O_i. */
+ * The workspace holds the fp32 dQ accumulator and the per-row D_i = dO_i . O_i.
+ * Errors as for st_attn_fwd. */
 ST_API st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void *o,
                         const float *lse, const void *dO, const st_layout_t *layout, void *dq,
                         void *dk, void *dv, void *workspace, size_t workspace_bytes,

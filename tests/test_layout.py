@@ -237,6 +237,10 @@ EXEC_SWEEP = [  # (family, mode, H, n, l, c) -- kernel-runnable layouts, every r
     (2, 2, 4, 768, 64, 16), (2, 4, 4, 384, 128, 128), (1, 1, 2, 3072, 64, 0),
     (1, 2, 2, 3072, 64, 0), (1, 1, 2, 32768, 256, 0), (2, 1, 2, 512, 128, 128),
     (2, 1, 6, 1024, 256, 128), (2, 3, 2, 512, 64, 16), (1, 1, 3, 384, 12, 0),
+    # edges: one tile (n = l = 128), l = 1 over one tile, summary runs of 1, 2 and 64 keys
+    # (128, 64 and 2 runs per compacted tile), merged fixed heads with c = 1, the 64-head maximum
+    (1, 1, 2, 128, 128, 0), (1, 2, 2, 128, 1, 0), (2, 1, 2, 128, 128, 1), (2, 1, 4, 512, 64, 1),
+    (2, 2, 2, 256, 128, 2), (2, 1, 2, 512, 128, 64), (2, 2, 2, 512, 64, 1), (2, 1, 64, 256, 128, 2),
 ]
 
 
