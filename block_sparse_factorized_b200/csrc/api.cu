@@ -1,6 +1,7 @@
 // api.cu -- C ABI entry points: argument checks, TMA descriptors, launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <string.h>
 
 #include <atomic>
@@ -65,29 +66,34 @@ bool encode(CUtensorMap *m, const void *base, CUtensorMapDataType dt, cuuint32_t
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor maps of a bf16 [BH, n, 64] tensor in the natural, grid-column and summary frames.
-bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum)
+// Tensor maps of a bf16 [BH, n, W] tensor in the natural, grid-column and summary frames.  A box
+// is 128 rows by one swizzle span of columns: W = 32 columns (64 bytes, 64-byte swizzle) or 64
+// columns (128 bytes, 128-byte swizzle); a 128-wide row is loaded as two boxes.
+bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum, int W = 64)
 {
     memset(&m, 0, sizeof(m));
-    const cuuint64_t row = 64 * 2, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
+    const cuuint64_t w = static_cast<cuuint64_t>(W), row = w * 2, n = static_cast<cuuint64_t>(g.n),
+                     l = static_cast<cuuint64_t>(g.l);
+    const cuuint32_t bx = static_cast<cuuint32_t>(W < 64 ? W : 64);
+    const CUtensorMapSwizzle swz = W < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     {
-        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[3] = {w, n, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[2] = {row, n * row};
-        const cuuint32_t box[3] = {64, 128, 1};
-        if (!encode(&m.nat, base, dt, 3, dims, str, box)) return false;
+        const cuuint32_t box[3] = {bx, 128, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box, swz)) return false;
     }
     if (col) {
-        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[4] = {w, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[3] = {l * row, row, n * row};
-        const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(g.Rt), static_cast<cuuint32_t>(g.cpt), 1};
-        if (!encode(&m.col, base, dt, 4, dims, str, box)) return false;
+        const cuuint32_t box[4] = {bx, static_cast<cuuint32_t>(g.Rt), static_cast<cuuint32_t>(g.cpt), 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box, swz)) return false;
     }
     if (sum) {
-        const cuuint64_t dims[4] = {64, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[4] = {w, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[3] = {row, l * row, n * row};
-        const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(g.c), static_cast<cuuint32_t>(g.upt), 1};
-        if (!encode(&m.sum, base, dt, 4, dims, str, box)) return false;
+        const cuuint32_t box[4] = {bx, static_cast<cuuint32_t>(g.c), static_cast<cuuint32_t>(g.upt), 1};
+        if (!encode(&m.sum, base, dt, 4, dims, str, box, swz)) return false;
     }
     return true;
 }
@@ -178,10 +184,15 @@ Frames frames_used(const st_layout &L)
     return f;
 }
 
-// Row widths the kernels are built for: query-key and value rows of 64 elements.
-bool widths_supported(const st_desc_t *desc)
+int64_t value_width(const st_desc_t *desc) { return desc->dv == 0 ? desc->d : desc->dv; }
+
+// Row widths the kernels are built for.  The bf16 forward: (query-key, value) = (32, 32),
+// (64, 64), (128, 128), (64, 128).  Everything else: 64 and 64.
+bool widths_supported(const st_desc_t *desc, bool fwd = false)
 {
-    const int64_t dv = desc->dv == 0 ? desc->d : desc->dv;
+    const int64_t dv = value_width(desc);
+    if (fwd && desc->dtype == ST_BF16 && desc->d <= 128 && dv <= 128)
+        return st::fwd_bf16_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv));
     return desc->d == 64 && dv == 64;
 }
 
@@ -194,14 +205,14 @@ bool sizes_valid(const st_desc_t *desc)
            desc->batch * desc->heads <= (1ll << 40) / desc->n;
 }
 
-st_status_t check_common(const st_layout *L, const st_desc_t *desc)
+st_status_t check_common(const st_layout *L, const st_desc_t *desc, bool fwd = false)
 {
     if (!L || !desc) return ST_ERR_INVALID_ARG;
     if (!sizes_valid(desc)) return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L->pat.num_heads || desc->n != L->n) return ST_ERR_INVALID_ARG;
     if (!L->exec_ok) return ST_ERR_UNSUPPORTED;
-    if (!widths_supported(desc)) return ST_ERR_UNSUPPORTED;
+    if (!widths_supported(desc, fwd)) return ST_ERR_UNSUPPORTED;
     if (desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
     if (!L->uploaded) return ST_ERR_NOT_UPLOADED;
     int dev = -1;
@@ -258,7 +269,7 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
                         const st_desc_t *desc, st_stream_t stream)
 {
     if (!q || !k || !v || !o || !lse) return ST_ERR_INVALID_ARG;
-    const st_status_t cs = check_common(layout, desc);
+    const st_status_t cs = check_common(layout, desc, true);
     if (cs != ST_OK) return cs;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ST_ERR_ALIGNMENT;
@@ -266,6 +277,7 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
     const int64_t BH = desc->batch * desc->heads;
     const Frames f = frames_used(L);
     const bool f32 = desc->dtype == ST_FP32;
+    const int dqk = static_cast<int>(desc->d), dv = static_cast<int>(value_width(desc));
     st::FwdParams p;
     memset(&p, 0, sizeof(p));
     if (!workspace || workspace_bytes < st_attn_fwd_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
@@ -285,15 +297,16 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
             return ST_ERR_CUDA;
         p.o_f32 = static_cast<float *>(o);
         p.o_prev_f32 = static_cast<const float *>(o);
-    } else if (!make_maps(p.q, q, L.geom, BH, f.qcol, false) || !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum) ||
-               !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum)) {
+    } else if (!make_maps(p.q, q, L.geom, BH, f.qcol, false, dqk) ||
+               !make_maps(p.k, k, L.geom, BH, f.kcol, f.ksum, dqk) ||
+               !make_maps(p.v, v, L.geom, BH, f.kcol, f.ksum, dv)) {
         return ST_ERR_CUDA;
     }
     p.parts = L.d_parts;
     p.batch = static_cast<int32_t>(desc->batch);
     p.heads = static_cast<int32_t>(desc->heads);
     p.g = L.geom;
-    p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
+    p.scale_log2 = LOG2E / sqrtf(static_cast<float>(dqk));  // log2(e) / sqrt(d)
     p.lse = lse;
     if (!f32) p.o = static_cast<uint16_t *>(o);
     p.o_prev = static_cast<const uint16_t *>(o);
@@ -302,7 +315,7 @@ st_status_t st_attn_fwd(const void *q, const void *k, const void *v, const st_la
         p.items = L.d_fwd[pass];
         p.nitems = static_cast<int32_t>(L.fwd_items[pass].size());
         p.sched = sched + pass;
-        if (st::launch_fwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
+        if (st::launch_fwd(p, f32, dqk, dv, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
     return ST_OK;
 }
@@ -500,7 +513,8 @@ size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *
 {
     if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t nsplit = static_cast<size_t>((desc->n + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
-    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * st::DEC_PART * sizeof(float));
+    const size_t part = static_cast<size_t>(value_width(desc)) + 4;  // dec_part(dv) floats per chunk
+    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * part * sizeof(float));
 }
 
 st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache, const st_layout_t *layout,
@@ -512,7 +526,10 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     if (!sizes_valid(desc)) return ST_ERR_INVALID_ARG;
     if (desc->dtype != ST_BF16 && desc->dtype != ST_FP32) return ST_ERR_INVALID_ARG;
     if (desc->heads != L.pat.num_heads || desc->n != L.n || pos < 0 || pos >= L.n) return ST_ERR_INVALID_ARG;
-    if (!widths_supported(desc) || desc->heads > 64 || desc->batch * desc->heads > (1ll << 30)) return ST_ERR_UNSUPPORTED;
+    const int64_t dv = value_width(desc);
+    if (desc->d > 128 || dv > 128 || !st::decode_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv)) ||
+        desc->heads > 64 || desc->batch * desc->heads > (1ll << 30))
+        return ST_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
         return ST_ERR_ALIGNMENT;
     if (!workspace || workspace_bytes < st_attn_decode_workspace_bytes(desc, layout)) return ST_ERR_WORKSPACE;
@@ -538,10 +555,11 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     p.c = L.c;
     p.bh = static_cast<int32_t>(desc->batch * desc->heads);
     p.heads = static_cast<int32_t>(desc->heads);
-    p.scale_log2 = LOG2E / 8.0f;  // log2(e) / sqrt(64)
+    p.scale_log2 = LOG2E / sqrtf(static_cast<float>(desc->d));  // log2(e) / sqrt(d)
     const int64_t nsplit = (most + st::DEC_CHUNK - 1) / st::DEC_CHUNK;
     if (nsplit > 65535) return ST_ERR_UNSUPPORTED;  // grid dimension y: a row with over 4 M allowed keys
-    return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, stream) == cudaSuccess
+    return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, static_cast<int>(desc->d),
+                             static_cast<int>(dv), stream) == cudaSuccess
                ? ST_OK
                : ST_ERR_CUDA;
 }

@@ -11,11 +11,11 @@
 //
 // Every allowed set is a grid of runs followed by a contiguous range (KeySet, decode.h).  The keys of one
 // (batch, head) are split into chunks of DEC_CHUNK = 64 over the CTAs of grid row y; a CTA of 128
-// threads works as 16 groups of 8 lanes, a group taking 4 keys with each lane holding 8 of the 64
-// components (one 16-byte load per lane per bf16 row).  All K and V loads of a chunk are issued
-// before any is used (the work is one round trip to memory, not a chain of them); then scores,
-// their maximum and 2^(s - M) v.  Each CTA leaves (M, L, O) of its chunk in the workspace; a second
-// kernel combines the chunks of a (batch, head) by log-sum-exp weights.
+// threads works as 16 groups of 8 lanes, a group taking 4 keys with each lane holding an eighth of
+// the query-key row (d / 8 components) and of the value row (dv / 8).  All K and V loads of a chunk
+// are issued before any is used (the work is one round trip to memory, not a chain of them); then
+// scores, their maximum and 2^(s - M) v.  Each CTA leaves (M, L, O) of its chunk in the workspace; a
+// second kernel combines the chunks of a (batch, head) by log-sum-exp weights.
 #include "decode.h"
 #include "tiles.cuh"
 
@@ -25,30 +25,44 @@ namespace {
 constexpr int DEC_THREADS = 128;
 constexpr int DEC_GROUPS = DEC_THREADS / 8;
 
-template <bool F32>
-__device__ __forceinline__ void load8(const void *base, int64_t row, int lane8, float (&x)[8])
+// Elements N * lane8 .. N * lane8 + N - 1 of row `row` of a [rows, W] tensor, widened to fp32
+// (N = W / 8: 4, 8 or 16 elements, one to four 8- or 16-byte loads).
+template <bool F32, int W>
+__device__ __forceinline__ void load_part(const void *base, int64_t row, int lane8, float (&x)[W / 8])
 {
+    constexpr int N = W / 8;
     if (F32) {
-        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + row * 64 + 8 * lane8);
-        const float4 a = p[0], b = p[1];
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-    } else {
-        const uint4 a = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + row * 64 + 8 * lane8);
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + row * W + N * lane8);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            x[2 * e] = bf16_lo(w[e]);
-            x[2 * e + 1] = bf16_hi(w[e]);
+        for (int e = 0; e < N / 4; ++e) {
+            const float4 a = p[e];
+            x[4 * e] = a.x; x[4 * e + 1] = a.y; x[4 * e + 2] = a.z; x[4 * e + 3] = a.w;
+        }
+    } else if (N == 4) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(base) + row * W + N * lane8);
+        x[0] = bf16_lo(a.x); x[1] = bf16_hi(a.x); x[2] = bf16_lo(a.y); x[3] = bf16_hi(a.y);
+    } else {
+        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + row * W + N * lane8);
+#pragma unroll
+        for (int e = 0; e < N / 8; ++e) {
+            const uint4 a = p[e];
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                x[8 * e + 2 * t] = bf16_lo(w[t]);
+                x[8 * e + 2 * t + 1] = bf16_hi(w[t]);
+            }
         }
     }
 }
 
-template <bool F32>
+template <bool F32, int D, int DV>
 __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams p)
 {
     constexpr int KPG = DEC_CHUNK / DEC_GROUPS;  // keys per group
-    __shared__ float red[DEC_GROUPS][65];
+    constexpr int NQ = D / 8, NV = DV / 8;       // components per lane
+    constexpr int PART = dec_part(DV);
+    __shared__ float red[DEC_GROUPS][DV + 1];
     __shared__ float wmax[DEC_THREADS / 32];
     const int32_t bh = blockIdx.x, h = bh % p.heads;
     const KeySet ks = key_set(p.kind[h], p.pos, p.l, p.c, p.off[h]);
@@ -56,13 +70,13 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams 
     const int64_t e0 = static_cast<int64_t>(blockIdx.y) * DEC_CHUNK;
     const int grp = threadIdx.x >> 3, l8 = threadIdx.x & 7;
     const size_t cache = static_cast<size_t>(bh) * p.n;  // first cache row of this (batch, head)
-    float q[8];
-    load8<F32>(p.q, bh, l8, q);
+    float q[NQ];
+    load_part<F32, D>(p.q, bh, l8, q);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] *= p.scale_log2;  // scores in log2 units
+    for (int e = 0; e < NQ; ++e) q[e] *= p.scale_log2;  // scores in log2 units
     // The group's keys e0 + grp + 16 r (r < KPG): every K and V load first, so that one round trip
     // to memory serves the whole chunk.
-    float k[KPG][8], v[KPG][8];
+    float k[KPG][NQ], v[KPG][NV];
     bool valid[KPG];
 #pragma unroll
     for (int r = 0; r < KPG; ++r) {
@@ -70,8 +84,8 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams 
         valid[r] = e < total;
         if (valid[r]) {
             const int64_t row = cache + key_at(ks, e);
-            load8<F32>(p.k, row, l8, k[r]);
-            load8<F32>(p.v, row, l8, v[r]);
+            load_part<F32, D>(p.k, row, l8, k[r]);
+            load_part<F32, DV>(p.v, row, l8, v[r]);
         }
     }
     // scores (every lane runs every shuffle: the groups of a warp share them) and their maximum
@@ -81,7 +95,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams 
         float x = 0.f;
         if (valid[r])
 #pragma unroll
-            for (int t = 0; t < 8; ++t) x = fmaf(q[t], k[r][t], x);
+            for (int t = 0; t < NQ; ++t) x = fmaf(q[t], k[r][t], x);
         x += __shfl_xor_sync(0xffffffffu, x, 1);
         x += __shfl_xor_sync(0xffffffffu, x, 2);
         x += __shfl_xor_sync(0xffffffffu, x, 4);
@@ -94,68 +108,87 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams 
     __syncthreads();
     const float M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
     // sum of 2^(s - M) and of 2^(s - M) v (every lane of a group adds the same weight)
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, lsum = 0.f;
+    float acc[NV], lsum = 0.f;
+#pragma unroll
+    for (int t = 0; t < NV; ++t) acc[t] = 0.f;
 #pragma unroll
     for (int r = 0; r < KPG; ++r)
         if (valid[r]) {
             const float w = ex2(s[r] - M);
             lsum += w;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) acc[t] = fmaf(w, v[r][t], acc[t]);
+            for (int t = 0; t < NV; ++t) acc[t] = fmaf(w, v[r][t], acc[t]);
         }
 #pragma unroll
-    for (int t = 0; t < 8; ++t) red[grp][8 * l8 + t] = acc[t];
-    if (l8 == 0) red[grp][64] = lsum;
+    for (int t = 0; t < NV; ++t) red[grp][NV * l8 + t] = acc[t];
+    if (l8 == 0) red[grp][DV] = lsum;
     __syncthreads();
-    float *part = p.part + (static_cast<size_t>(bh) * gridDim.y + blockIdx.y) * DEC_PART;
-    if (threadIdx.x < 65) {
+    float *part = p.part + (static_cast<size_t>(bh) * gridDim.y + blockIdx.y) * PART;
+    for (int c = threadIdx.x; c < DV + 1; c += DEC_THREADS) {
         float sum = 0.f;
-        for (int g = 0; g < DEC_GROUPS; ++g) sum += red[g][threadIdx.x];  // fixed order
-        part[2 + threadIdx.x] = sum;  // O (64 columns) then L
+        for (int g = 0; g < DEC_GROUPS; ++g) sum += red[g][c];  // fixed order
+        part[2 + c] = sum;  // O (DV columns) then L
     }
     if (threadIdx.x == 0) part[0] = M;  // -inf for a chunk without keys
 }
 
 // One (batch, head) per CTA, one output column per thread: O = sum_c 2^(M_c - M) O_c / L,
 // L = sum_c 2^(M_c - M) L_c, lse = (M + log2 L) ln 2; a row without keys gets O = 0, lse = -inf.
-template <bool F32>
-__global__ void __launch_bounds__(64) decode_combine_kernel(const DecodeParams p, int32_t nsplit)
+template <bool F32, int DV>
+__global__ void __launch_bounds__(DV) decode_combine_kernel(const DecodeParams p, int32_t nsplit)
 {
+    constexpr int PART = dec_part(DV);
     const int32_t bh = blockIdx.x, t = threadIdx.x;
-    const float *part = p.part + static_cast<size_t>(bh) * nsplit * DEC_PART;
+    const float *part = p.part + static_cast<size_t>(bh) * nsplit * PART;
     float M = -INFINITY;
-    for (int c = 0; c < nsplit; ++c) M = fmaxf(M, part[c * DEC_PART]);
+    for (int c = 0; c < nsplit; ++c) M = fmaxf(M, part[c * PART]);
     float L = 0.f, o = 0.f;
     if (M != -INFINITY)
         for (int c = 0; c < nsplit; ++c) {
-            const float mc = part[c * DEC_PART];
+            const float mc = part[c * PART];
             const float w = mc == -INFINITY ? 0.f : ex2(mc - M);
-            L = fmaf(w, part[c * DEC_PART + 2 + 64], L);
-            o = fmaf(w, part[c * DEC_PART + 2 + t], o);
+            L = fmaf(w, part[c * PART + 2 + DV], L);
+            o = fmaf(w, part[c * PART + 2 + t], o);
         }
     const bool has = L > 0.f;
     o = has ? o / L : 0.f;
     if (F32)
-        static_cast<float *>(p.o)[static_cast<size_t>(bh) * 64 + t] = o;
+        static_cast<float *>(p.o)[static_cast<size_t>(bh) * DV + t] = o;
     else
-        static_cast<uint16_t *>(p.o)[static_cast<size_t>(bh) * 64 + t] =
+        static_cast<uint16_t *>(p.o)[static_cast<size_t>(bh) * DV + t] =
             static_cast<uint16_t>(pack_bf16(o, 0.f) & 0xFFFFu);
     if (t == 0) p.lse[bh] = has ? (M + lg2(L)) * LN2 : -INFINITY;
 }
 
-}  // namespace
-
-cudaError_t launch_decode(const DecodeParams &p, int32_t nsplit, bool f32, cudaStream_t s)
+template <bool F32, int D, int DV>
+cudaError_t launch_w(const DecodeParams &p, int32_t nsplit, cudaStream_t s)
 {
     const dim3 grid(static_cast<unsigned>(p.bh), static_cast<unsigned>(nsplit));
-    if (f32) {
-        decode_kernel<true><<<grid, DEC_THREADS, 0, s>>>(p);
-        decode_combine_kernel<true><<<static_cast<unsigned>(p.bh), 64, 0, s>>>(p, nsplit);
-    } else {
-        decode_kernel<false><<<grid, DEC_THREADS, 0, s>>>(p);
-        decode_combine_kernel<false><<<static_cast<unsigned>(p.bh), 64, 0, s>>>(p, nsplit);
-    }
+    decode_kernel<F32, D, DV><<<grid, DEC_THREADS, 0, s>>>(p);
+    decode_combine_kernel<F32, DV><<<static_cast<unsigned>(p.bh), DV, 0, s>>>(p, nsplit);
     return cudaGetLastError();
+}
+
+template <bool F32>
+cudaError_t launch_f(const DecodeParams &p, int32_t nsplit, int d, int dv, cudaStream_t s)
+{
+    if (d == 32 && dv == 32) return launch_w<F32, 32, 32>(p, nsplit, s);
+    if (d == 64 && dv == 64) return launch_w<F32, 64, 64>(p, nsplit, s);
+    if (d == 128 && dv == 128) return launch_w<F32, 128, 128>(p, nsplit, s);
+    if (d == 64 && dv == 128) return launch_w<F32, 64, 128>(p, nsplit, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool decode_widths_supported(int d, int dv)
+{
+    return (d == dv && (d == 32 || d == 64 || d == 128)) || (d == 64 && dv == 128);
+}
+
+cudaError_t launch_decode(const DecodeParams &p, int32_t nsplit, bool f32, int d, int dv, cudaStream_t s)
+{
+    return f32 ? launch_f<true>(p, nsplit, d, dv, s) : launch_f<false>(p, nsplit, d, dv, s);
 }
 
 }  // namespace st

@@ -8,7 +8,8 @@
 namespace st {
 
 constexpr int DEC_CHUNK = 64;   // keys per CTA (16 groups x 4 keys)
-constexpr int DEC_PART = 68;    // floats per chunk result: M, (unused), O[64], L, (pad)
+// floats per chunk result for value rows of width dv: M, (unused), O[dv], L, (pad)
+__host__ __device__ constexpr int dec_part(int dv) { return dv + 4; }
 
 // Allowed keys of one row: nu runs, run u covering g0 + u * gs .. + glen - 1 (the last run cut to
 // glast keys), and the range r0 .. r0 + nr - 1.  Runs and range are disjoint and every run lies
@@ -84,17 +85,20 @@ ST_HD int64_t key_at(const KeySet &k, int64_t e)
 }
 
 struct DecodeParams {
-    const void *q;      // [B*H, 64] one query row per (batch, head)
-    const void *k, *v;  // [B*H, n, 64] caches (rows past pos unread)
-    void *o;            // [B*H, 64]
+    const void *q;      // [B*H, d] one query row per (batch, head)
+    const void *k;      // [B*H, n, d] key cache (rows past pos unread)
+    const void *v;      // [B*H, n, dv] value cache (rows past pos unread)
+    void *o;            // [B*H, dv]
     float *lse;         // [B*H], natural log
-    float *part;        // [B*H, nsplit, DEC_PART] chunk results (workspace)
+    float *part;        // [B*H, nsplit, dec_part(dv)] chunk results (workspace)
     int32_t kind[64], off[64];
     int64_t pos, n, l, c;
     int32_t bh, heads;
-    float scale_log2;   // log2(e) / sqrt(64)
+    float scale_log2;   // log2(e) / sqrt(d)
 };
 
-cudaError_t launch_decode(const DecodeParams &p, int32_t nsplit, bool f32, cudaStream_t s);
+// Row widths (query-key d, value dv) with a decode kernel: (32, 32), (64, 64), (128, 128), (64, 128).
+bool decode_widths_supported(int d, int dv);
+cudaError_t launch_decode(const DecodeParams &p, int32_t nsplit, bool f32, int d, int dv, cudaStream_t s);
 
 }  // namespace st

@@ -555,9 +555,10 @@ cudaError_t launch_fwd_split(const FwdParams &p, cudaStream_t s)
 
 }  // namespace
 
-cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s)
+cudaError_t launch_fwd(const FwdParams &p, bool split, int dqk, int dv, cudaStream_t s)
 {
-    return split ? launch_fwd_split(p, s) : launch_fwd_bf16(p, s);
+    if (split) return (dqk == 64 && dv == 64) ? launch_fwd_split(p, s) : cudaErrorInvalidValue;
+    return launch_fwd_bf16(p, dqk, dv, s);
 }
 
 }  // namespace st

@@ -27,24 +27,68 @@
 namespace st {
 namespace {
 
+// Per-width tile geometry.  A 128-row bf16 tile of W columns is loaded as NBOX TMA boxes of BOX
+// columns, each one swizzle span wide (64-byte swizzle for W = 32, 128-byte otherwise), stored
+// one after another: box b holds columns b*BOX .. b*BOX + BOX - 1 of every row.
+template <int W>
+struct Tile {
+    static_assert(W == 32 || W == 64 || W == 128, "row width");
+    static constexpr int BOX = W < 64 ? W : 64;
+    static constexpr int NBOX = W / BOX;
+    static constexpr uint32_t SPAN = BOX * 2;                // bytes per row of a box (swizzle span)
+    static constexpr uint32_t BOX_BYTES = 128 * SPAN;
+    static constexpr uint32_t BYTES = NBOX * BOX_BYTES;
+    static constexpr uint32_t LAYOUT = W < 64 ? UMMA_SW64 : UMMA_SW128;
+    // K-major operand (rows = M or N, K = the W columns): the K16 step k starts 32 bytes further
+    // in the same box, or in the next box once a box's columns are used up; 8-row groups are
+    // 8 * SPAN bytes apart.
+    __device__ static uint64_t kmajor(uint32_t base, int k)
+    {
+        const int col = 16 * k;
+        return desc_swz(base + (col / BOX) * BOX_BYTES + (col % BOX) * 2, 16, 8 * SPAN, LAYOUT);
+    }
+    // MN-major operand (K = the 128 rows, N = the W columns): the K16 step k starts 16 rows
+    // further; 8-row groups are 8 * SPAN bytes apart (SBO) and the N atoms are the boxes (LBO).
+    __device__ static uint64_t mnmajor(uint32_t base, int k)
+    {
+        return desc_swz(base + 16 * k * SPAN, BOX_BYTES, 8 * SPAN, LAYOUT);
+    }
+};
+
+// TMA load of tile t of frame fr of batch-head bh into dst: NBOX boxes, one transaction count.
+template <int W>
+__device__ __forceinline__ void load_tile_w(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o, int32_t t,
+                                            int32_t bh, uint8_t *dst, uint64_t *bar)
+{
+#pragma unroll
+    for (int b = 0; b < Tile<W>::NBOX; ++b)
+        load_tile_x(m, fr, g, o, t, bh, b * Tile<W>::BOX, dst + b * Tile<W>::BOX_BYTES, bar);
+}
+
 constexpr int NST = 2;                         // K/V ring depth
 constexpr int NQB = 2;                         // Q buffers
 constexpr int NSCHED = 4;                      // claimed-unit ring depth
-constexpr uint32_t TB = TILE_BYTES;            // one 128 x 64 bf16 tile, 16 KB
 constexpr int THREADS = 192;
-constexpr int CTAS_PER_SM = 2;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_S = 0;                  // S: 128 fp32 columns
-constexpr uint32_t COL_O = 128;                // O: 64 fp32 columns
-constexpr uint32_t COL_P = 192;                // P: 128 bf16 as 64 columns of pairs
 constexpr float RESCALE_LOG2 = 8.0f;           // keep a stale max while it is within 2^8
 
-constexpr uint32_t OFF_Q = 0;                  // NQB tiles
-constexpr uint32_t OFF_K = OFF_Q + NQB * TB;   // NST tiles
-constexpr uint32_t OFF_V = OFF_K + NST * TB;   // NST tiles
-constexpr uint32_t OFF_BAR = OFF_V + NST * TB;
-constexpr uint32_t OFF_UNITS = OFF_BAR + 256;  // the claimed units' fields, NSCHED entries
-constexpr uint32_t SMEM_BYTES = OFF_UNITS + NSCHED * 96;
+// Query-key rows of width DQK, value rows of width DV.
+template <int DQK, int DV>
+struct Cfg {
+    static constexpr uint32_t QB = Tile<DQK>::BYTES, VB = Tile<DV>::BYTES;
+    static constexpr uint32_t COL_S = 0;                       // S: 128 fp32 columns
+    static constexpr uint32_t COL_O = 128;                     // O: DV fp32 columns
+    static constexpr uint32_t COL_P = 128 + DV;                // P: 128 bf16 as 64 columns of pairs
+    static constexpr uint32_t COLS_USED = COL_P + 64;
+    static constexpr int CTAS_PER_SM = COLS_USED <= 256 ? 2 : 1;
+    static constexpr uint32_t TMEM_COLS = CTAS_PER_SM == 2 ? 256 : 512;
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_K = OFF_Q + NQB * QB;
+    static constexpr uint32_t OFF_V = OFF_K + NST * QB;
+    static constexpr uint32_t OFF_BAR = OFF_V + NST * VB;
+    static constexpr uint32_t OFF_UNITS = OFF_BAR + 256;
+    static constexpr uint32_t SMEM_BYTES = OFF_UNITS + 4 * 96;
+    static_assert(SMEM_BYTES * CTAS_PER_SM <= 228 * 1024 - CTAS_PER_SM * 1024, "shared memory per SM");
+};
 
 struct Bars {
     uint64_t q_full[NQB], q_empty[NQB];
@@ -112,8 +156,13 @@ __device__ __forceinline__ uint32_t (&part32(uint32_t (&v)[128], int e))[32]
     return *reinterpret_cast<uint32_t(*)[32]>(&v[e]);
 }
 
-__global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __grid_constant__ FwdParams p)
+template <int DQK, int DV>
+__global__ void __launch_bounds__(THREADS, (Cfg<DQK, DV>::CTAS_PER_SM)) fwd_bf16_kernel(const __grid_constant__ FwdParams p)
 {
+    using C = Cfg<DQK, DV>;
+    constexpr uint32_t OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_BAR = C::OFF_BAR,
+                       OFF_UNITS = C::OFF_UNITS, QB = C::QB, VB = C::VB, TMEM_COLS = C::TMEM_COLS,
+                       COL_S = C::COL_S, COL_O = C::COL_O, COL_P = C::COL_P;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BAR);
@@ -173,16 +222,16 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
             auto load_k = [&](const Unit &U, int32_t tile) {
                 const int s = TK % NST;
                 if (TK >= NST && !mbar_wait(&bars->k_empty[s], ((TK / NST) - 1) & 1, abort, p.err)) return false;
-                mbar_arrive_expect_tx(&bars->k_full[s], TB);
-                load_tile(p.k, U.part.kframe, p.g, U.part.o, tile, U.bh, smem + OFF_K + s * TB, &bars->k_full[s]);
+                mbar_arrive_expect_tx(&bars->k_full[s], QB);
+                load_tile_w<DQK>(p.k, U.part.kframe, p.g, U.part.o, tile, U.bh, smem + OFF_K + s * QB, &bars->k_full[s]);
                 ++TK;
                 return true;
             };
             auto load_v = [&](const Unit &U, int32_t tile) {
                 const int s = TV % NST;
                 if (TV >= NST && !mbar_wait(&bars->v_empty[s], ((TV / NST) - 1) & 1, abort, p.err)) return false;
-                mbar_arrive_expect_tx(&bars->v_full[s], TB);
-                load_tile(p.v, U.part.kframe, p.g, U.part.o, tile, U.bh, smem + OFF_V + s * TB, &bars->v_full[s]);
+                mbar_arrive_expect_tx(&bars->v_full[s], VB);
+                load_tile_w<DV>(p.v, U.part.kframe, p.g, U.part.o, tile, U.bh, smem + OFF_V + s * VB, &bars->v_full[s]);
                 ++TV;
                 return true;
             };
@@ -206,8 +255,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
                 const int qb = kq % NQB;
                 if (kq >= NQB && !mbar_wait(&bars->q_empty[qb], ((kq / NQB) - 1) & 1, abort, p.err)) break;
                 ++kq;
-                mbar_arrive_expect_tx(&bars->q_full[qb], TB);
-                load_tile(p.q, U.part.qframe, p.g, U.part.o, U.w.tile, U.bh, smem + OFF_Q + qb * TB, &bars->q_full[qb]);
+                mbar_arrive_expect_tx(&bars->q_full[qb], QB);
+                load_tile_w<DQK>(p.q, U.part.qframe, p.g, U.part.o, U.w.tile, U.bh, smem + OFF_Q + qb * QB, &bars->q_full[qb]);
                 fail = !load_k(U, U.w.begin);
                 for (int it = 0; !fail && it < U.nkt; ++it)
                     fail = (it + 1 < U.nkt && !load_k(U, U.w.begin + it + 1)) || !load_v(U, U.w.begin + it);
@@ -226,24 +275,24 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
         // ---------------- MMA issuer ----------------
         if (lane == 0 && run) {
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idO = idesc_bf16(128, 64, false, true);
-            // S = Q K^T: both operands K-major, 16 elements (32 bytes) of d per step
+            constexpr uint32_t idO = idesc_bf16(128, DV, false, true);
+            // S = Q K^T: both operands K-major, DQK / 16 steps of 16 elements
             auto issue_s = [&](int32_t t, int qb) {
-                const uint32_t sQ = smem_u32(smem + OFF_Q + qb * TB), sK = smem_u32(smem + OFF_K + (t % NST) * TB);
+                const uint32_t sQ = smem_u32(smem + OFF_Q + qb * QB), sK = smem_u32(smem + OFF_K + (t % NST) * QB);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ss(tbase + COL_S, desc_sw128(sQ + 32 * k, 16, 1024), desc_sw128(sK + 32 * k, 16, 1024),
-                                idS, k > 0 ? 1u : 0u);
+                for (int k = 0; k < DQK / 16; ++k)
+                    mma_bf16_ss(tbase + COL_S, Tile<DQK>::kmajor(sQ, k), Tile<DQK>::kmajor(sK, k), idS,
+                                k > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full);
                 mma_commit(&bars->k_empty[t % NST]);
             };
             // O += P V: P from TMEM (8 columns of bf16 pairs = 16 keys per step), V MN-major
-            // (16 keys = 2048 bytes per step); the first tile of a unit overwrites O
+            // (16 keys per step); the first tile of a unit overwrites O
             auto issue_pv = [&](int32_t t, bool first) {
-                const uint32_t sV = smem_u32(smem + OFF_V + (t % NST) * TB);
+                const uint32_t sV = smem_u32(smem + OFF_V + (t % NST) * VB);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16_ts(tbase + COL_O, tbase + COL_P + 8 * k, desc_sw128(sV + k * 2048, TB, 1024), idO,
+                    mma_bf16_ts(tbase + COL_O, tbase + COL_P + 8 * k, Tile<DV>::mnmajor(sV, k), idO,
                                 (!first || k > 0) ? 1u : 0u);
                 mma_commit(&bars->pv_done);
                 mma_commit(&bars->v_empty[t % NST]);
@@ -326,8 +375,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
                     return;
                 }
                 tc_fence_after();
-                tmem_ld32(tO, part32(v, 0));
-                tmem_ld32(tO + 32, part32(v, 32));
+#pragma unroll
+                for (int c = 0; c < DV / 32; ++c) tmem_ld32(tO + 32 * c, part32(v, 32 * c));
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bars->o_free);  // the next unit's first product may now overwrite O
@@ -350,27 +399,27 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
                 }
             }
             if (e.i < 0 || *abort != 0) return;  // grid-frame padding row
-            float acc[64];
+            // 8 columns (16 bytes) at a time; a merge reads each 16 bytes of the first pass's row
+            // before it overwrites them
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * DV);
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + rowoff * DV);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) acc[c] = has_o ? cnew * __uint_as_float(v[c]) : 0.f;
-            if (cprev != 0.f) {  // this thread reads the first pass's row before overwriting it
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * 64);
+            for (int q = 0; q < DV / 8; ++q) {
+                float a[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int c = 0; c < 8; ++c) a[c] = has_o ? cnew * __uint_as_float(v[8 * q + c]) : 0.f;
+                if (cprev != 0.f) {
                     const uint4 x = src[q];
                     const uint32_t pw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        acc[8 * q + 2 * c] = fmaf(cprev, bf16_lo(pw[c]), acc[8 * q + 2 * c]);
-                        acc[8 * q + 2 * c + 1] = fmaf(cprev, bf16_hi(pw[c]), acc[8 * q + 2 * c + 1]);
+                        a[2 * c] = fmaf(cprev, bf16_lo(pw[c]), a[2 * c]);
+                        a[2 * c + 1] = fmaf(cprev, bf16_hi(pw[c]), a[2 * c + 1]);
                     }
                 }
+                dst[q] = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                                    pack_bf16(a[6], a[7]));
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + rowoff * 64);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[q] = make_uint4(pack_bf16(acc[8 * q], acc[8 * q + 1]), pack_bf16(acc[8 * q + 2], acc[8 * q + 3]),
-                                    pack_bf16(acc[8 * q + 4], acc[8 * q + 5]), pack_bf16(acc[8 * q + 6], acc[8 * q + 7]));
             p.lse[rowoff] = lse2 * LN2;
         };
         for (int32_t j = 0; ok; ++j) {
@@ -431,7 +480,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
                 if (t > 0) tc_fence_after();
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < DV / 32; ++c) {
                         uint32_t o[32];
                         tmem_ld32(tO + 32 * c, o);
                         tmem_wait_ld();
@@ -467,21 +516,40 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) fwd_bf16_kernel(const __
     }
 }
 
-}  // namespace
 
-cudaError_t launch_fwd_bf16(const FwdParams &p, cudaStream_t s)
+template <int DQK, int DV>
+cudaError_t launch_w(const FwdParams &p, cudaStream_t s)
 {
+    using C = Cfg<DQK, DV>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const int64_t units = static_cast<int64_t>(p.nitems) * p.batch;
     if (units == 0) return cudaSuccess;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * CTAS_PER_SM;
-    fwd_bf16_kernel<<<static_cast<unsigned>(units < cap ? units : cap), THREADS, SMEM_BYTES, s>>>(p);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * C::CTAS_PER_SM;
+    fwd_bf16_kernel<DQK, DV><<<static_cast<unsigned>(units < cap ? units : cap), THREADS, C::SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// Row widths (query-key, value) with a kernel: (32, 32), (64, 64), (128, 128), (64, 128).
+bool fwd_bf16_widths_supported(int dqk, int dv)
+{
+    return (dqk == dv && (dqk == 32 || dqk == 64 || dqk == 128)) || (dqk == 64 && dv == 128);
+}
+
+cudaError_t launch_fwd_bf16(const FwdParams &p, int dqk, int dv, cudaStream_t s)
+{
+    if (dqk == 32 && dv == 32) return launch_w<32, 32>(p, s);
+    if (dqk == 64 && dv == 64) return launch_w<64, 64>(p, s);
+    if (dqk == 128 && dv == 128) return launch_w<128, 128>(p, s);
+    if (dqk == 64 && dv == 128) return launch_w<64, 128>(p, s);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace st

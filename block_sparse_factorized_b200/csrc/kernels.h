@@ -103,8 +103,11 @@ struct SplitParams {
 // Streaming multiprocessors of the current device (queried once per device).
 int sm_count();
 
-cudaError_t launch_fwd(const FwdParams &p, bool split, cudaStream_t s);
-cudaError_t launch_fwd_bf16(const FwdParams &p, cudaStream_t s);
+// Forward launch: the split-precision kernel (fp32 I/O, 64-wide rows) or the bf16 kernel for
+// query-key rows of width dqk and value rows of width dv.
+cudaError_t launch_fwd(const FwdParams &p, bool split, int dqk, int dv, cudaStream_t s);
+cudaError_t launch_fwd_bf16(const FwdParams &p, int dqk, int dv, cudaStream_t s);
+bool fwd_bf16_widths_supported(int dqk, int dv);
 cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s);
 cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s);

@@ -281,19 +281,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-// UMMA shared-memory descriptor for a 128-byte-swizzled operand (rows of 128 B, 8-row
-// groups of 1024 B).  lbo/sbo in bytes.  Fields: start address >> 4 in bits [0,14), leading
-// byte offset >> 4 in [16,30), stride byte offset >> 4 in [32,46), descriptor version 1 in
-// [46,48), base offset 0, layout type SWIZZLE_128B (2) in [61,64).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+// UMMA shared-memory descriptor of a swizzled operand.  lbo/sbo in bytes.  Fields: start
+// address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30), stride byte offset >> 4 in
+// [32,46), descriptor version 1 in [46,48), base offset 0, layout type in [61,64): 2 for the
+// 128-byte swizzle (rows of 128 B, 8-row groups of 1024 B), 4 for the 64-byte swizzle (rows of
+// 64 B, 8-row groups of 512 B).
+constexpr uint32_t UMMA_SW128 = 2, UMMA_SW64 = 4;
+__device__ __forceinline__ uint64_t desc_swz(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
 {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
     d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;
-    d |= 2ull << 61;
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
     return d;
+}
+
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return desc_swz(saddr, lbo, sbo, UMMA_SW128);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.  a_mn / b_mn: operand stored

@@ -49,18 +49,26 @@ __device__ __forceinline__ const CUtensorMap *frame_map(const FrameMaps &m, int3
     return fr == FR_NAT ? &m.nat : (fr == FR_COL ? &m.col : &m.sum);
 }
 
+// TMA load of columns x .. x + box - 1 (the map's box width) of tile t of frame fr (summary
+// offset o) of batch-head bh into dst.
+__device__ __forceinline__ void load_tile_x(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o, int32_t t,
+                                            int32_t bh, int32_t x, void *dst, uint64_t *bar)
+{
+    if (fr == FR_NAT) {
+        tma_load_3d(dst, &m.nat, bar, x, t * TILE, bh);
+    } else if (fr == FR_COL) {
+        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
+        tma_load_4d(dst, &m.col, bar, x, rt * TILE, grp * g.cpt, bh);
+    } else {
+        tma_load_4d(dst, &m.sum, bar, x, g.l - g.c - o, t * g.upt, bh);
+    }
+}
+
 // TMA load of tile t of frame fr (summary offset o) of batch-head bh into dst (16 KB).
 __device__ __forceinline__ void load_tile(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
                                           int32_t t, int32_t bh, void *dst, uint64_t *bar)
 {
-    if (fr == FR_NAT) {
-        tma_load_3d(dst, &m.nat, bar, 0, t * TILE, bh);
-    } else if (fr == FR_COL) {
-        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
-        tma_load_4d(dst, &m.col, bar, 0, rt * TILE, grp * g.cpt, bh);
-    } else {
-        tma_load_4d(dst, &m.sum, bar, 0, g.l - g.c - o, t * g.upt, bh);
-    }
+    load_tile_x(m, fr, g, o, t, bh, 0, dst, bar);
 }
 
 // L2 prefetch of tile t of frame fr (same coordinates as load_tile).

@@ -91,8 +91,9 @@ typedef enum { ST_BF16 = 1, ST_FP32 = 2 } st_dtype_t;
 /* Shapes of one call.  Q, K, dQ, dK are [batch, heads, n, d]; V, O, dO, dV are
  * [batch, heads, n, dv] ("Sparse Transformers 深度解读报告" §4.5: the models' per-head widths
  * are 32, 64 and 128, and the CIFAR-10 model halves its query-key projection, d = dv / 2).
- * Scores are scaled by 1/sqrt(d).  The kernels handle d = dv = 64; other widths are valid
- * arguments and return ST_ERR_UNSUPPORTED. */
+ * Scores are scaled by 1/sqrt(d).  Widths with kernels: the forward (bf16) and the decode step
+ * take (d, dv) = (32, 32), (64, 64), (128, 128) and (64, 128); the backward pass and the fp32
+ * forward take (64, 64).  Other widths are valid arguments and return ST_ERR_UNSUPPORTED. */
 typedef struct {
     int64_t batch, heads, n, d; /* heads must equal the layout's num_heads, n its n */
     int32_t dtype;              /* st_dtype_t: Q, K, V, O, dO, dQ, dK, dV all in this type */

@@ -34,10 +34,11 @@ def positions(w, count=4, seed=0):
     return sorted(p for p in base if 0 <= p < w.n)
 
 
-def run_case(w, tol_scale=1.0):
+def run_case(w, with_fwd=True):
     (qd, kd, vd, _), (q, k, v, _) = cuda_inputs(w)
     lay = bsf.Layout(w.family, w.head_mode, w.heads, w.n, w.l, w.c, a2_offset_step=w.offset_step).upload()
-    o_fwd, lse_fwd = bsf.st_attn_fwd(qd, kd, vd, lay)
+    if with_fwd:
+        o_fwd, lse_fwd = bsf.st_attn_fwd(qd, kd, vd, lay)
     prob = problem_of(w)
     k64, v64 = to64(k), to64(v)
     for pos in positions(w):
@@ -49,8 +50,9 @@ def run_case(w, tol_scale=1.0):
         torch.cuda.synchronize()
         o_ref, lse_ref = prob.decode(to64(q[:, :, pos]), k64, v64, pos)
         check_o_lse(to64(o), to64(lse), o_ref, lse_ref, f"{w.name} pos {pos}")
-        check_o_lse(to64(o), to64(lse), to64(o_fwd[:, :, pos]), to64(lse_fwd[:, :, pos]),
-                    f"{w.name} pos {pos} vs forward row")
+        if with_fwd:
+            check_o_lse(to64(o), to64(lse), to64(o_fwd[:, :, pos]), to64(lse_fwd[:, :, pos]),
+                        f"{w.name} pos {pos} vs forward row")
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
@@ -76,3 +78,19 @@ def test_decode_empty_set_and_errors():
     for bad in (-1, w.n):
         with pytest.raises(bsf.StError):
             bsf.st_attn_decode(qd[:, :, 0].contiguous(), kd, vd, lay, bad)
+
+
+@pytest.mark.parametrize("d,dv", [(32, 32), (128, 128), (64, 128)], ids=lambda x: str(x))
+@pytest.mark.parametrize("w", [WORKLOADS["fixed_n12288_l128_c32"], WORKLOADS["strided_merged_n3072_l64"],
+                               Workload("f_merged_n4096_l128_c32", FIXED, MERGED, 4096, 128, 32, 2, 2)],
+                         ids=lambda w: w.name)
+def test_decode_widths(w, d, dv):
+    """Query-key rows of width d, value rows of width dv ("Sparse Transformers 深度解读报告" §4.5's
+    per-head widths): the decode step against the oracle's decode and the forward's row pos."""
+    run_case(w.with_(d=d, dv=dv))
+
+
+@pytest.mark.parametrize("d,dv", [(32, 32), (64, 128)], ids=lambda x: str(x))
+def test_decode_widths_fp32(d, dv):
+    """fp32 I/O at the other widths (the forward has no fp32 kernel there: oracle only)."""
+    run_case(FP32[0].with_(d=d, dv=dv), with_fwd=False)

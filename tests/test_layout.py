@@ -76,15 +76,19 @@ def test_argument_errors():
     fake = ctypes.c_void_p(1 << 20)
     d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 4
-    d = _abi.st_desc_t(1, 2, 256, 32, 1, 0)
-    assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 2
-    # value width: 0 or 64 pass the width check (NOT_UPLOADED next), other widths are valid but
-    # unsupported, a negative width is invalid
-    for dv, want in ((64, 4), (128, 2), (32, 2), (-1, 1)):
-        d = _abi.st_desc_t(1, 2, 256, 64, 1, dv)
-        assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == want
+    # row widths (query-key d, value dv; dv = 0 means d): the bf16 forward takes (32, 32),
+    # (64, 64), (128, 128) and (64, 128) -- those pass the width check and meet NOT_UPLOADED --
+    # the backward and fp32 I/O only (64, 64); other widths are valid but unsupported, a negative
+    # value width is invalid
+    for dqk, dv, dt, fwd_want, bwd_want in ((32, 0, 1, 4, 2), (128, 0, 1, 4, 2), (64, 128, 1, 4, 2),
+                                            (64, 64, 1, 4, 4), (64, 0, 2, 4, 4), (32, 0, 2, 2, 2),
+                                            (48, 0, 1, 2, 2), (64, 32, 1, 2, 2), (256, 0, 1, 2, 2),
+                                            (64, -1, 1, 1, 1)):
+        d = _abi.st_desc_t(1, 2, 256, dqk, dt, dv)
+        assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d),
+                               None) == fwd_want, (dqk, dv, dt)
         assert lib.st_attn_bwd(fake, fake, fake, fake, fake, fake, lay.handle, fake, fake, fake, None, 0,
-                               ctypes.byref(d), None) == want
+                               ctypes.byref(d), None) == bwd_want, (dqk, dv, dt)
     d = _abi.st_desc_t(1, 3, 256, 64, 1, 0)      # heads mismatch
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 1
     d = _abi.st_desc_t(1, 2, 256, 64, 7, 0)      # bad dtype
@@ -134,9 +138,13 @@ def test_decode_argument_errors():
     assert call(pos=-1) == 1 and call(pos=256) == 1   # position outside [0, n)
     assert call(desc=_abi.st_desc_t(1, 3, 256, 64, 1, 0)) == 1   # heads are not the layout's
     assert call(desc=_abi.st_desc_t(1, 2, 512, 64, 1, 0)) == 1   # n is not the layout's
-    assert call(desc=_abi.st_desc_t(1, 2, 256, 32, 1, 0)) == 2   # d != 64
-    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, 128)) == 2  # value width != 64
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, 32)) == 2   # no kernel for (64, 32)
+    assert call(desc=_abi.st_desc_t(1, 2, 256, 48, 1, 0)) == 2    # nor for 48-wide rows
     assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, -1)) == 1   # negative value width
+    # the chunk record is dv + 4 floats: 2 x 4 x 132 x 4 bytes at dv = 128
+    wide = _abi.st_desc_t(1, 2, 256, 64, 1, 128)
+    assert lib.st_attn_decode_workspace_bytes(ctypes.byref(wide), lay.handle) == 4352
+    assert call(desc=wide) == 8                                  # the 64-wide workspace is too small
     assert call(q=odd) == 3                       # misaligned
     assert call(w=None) == 8 and call(wb=need - 1) == 8          # workspace missing / too small
     keys = np.empty(256, dtype=np.int64)

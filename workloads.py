@@ -32,10 +32,11 @@ class Workload:
     c: int
     batch: int
     heads: int
-    d: int = 64
+    d: int = 64           # width of the query and key rows
     dtype: str = "bf16"  # "bf16" or "fp32"
     offset_step: int = 0  # fixed-pattern head-2 sub-block step (0: c)
     seed: int = 0
+    dv: int = 0           # width of the value (and output-gradient) rows; 0: d
 
     @property
     def torch_dtype(self):
@@ -43,6 +44,9 @@ class Workload:
 
     def shape(self):
         return (self.batch, self.heads, self.n, self.d)
+
+    def value_shape(self):
+        return (self.batch, self.heads, self.n, self.dv or self.d)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -75,11 +79,11 @@ def make_inputs(w: Workload, with_grad_out: bool = True):
     """Return (q, k, v, do) CPU tensors in the workload's dtype, drawn as described above."""
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
-    shp = w.shape()
+    shp, vshp = w.shape(), w.value_shape()
     q = torch.randn(shp, generator=g, dtype=torch.float32)
     k = torch.randn(shp, generator=g, dtype=torch.float32)
-    v = torch.randn(shp, generator=g, dtype=torch.float32)
-    do = torch.randn(shp, generator=g, dtype=torch.float32) if with_grad_out else None
+    v = torch.randn(vshp, generator=g, dtype=torch.float32)
+    do = torch.randn(vshp, generator=g, dtype=torch.float32) if with_grad_out else None
     dt = w.torch_dtype
     out = [q.to(dt), k.to(dt), v.to(dt)]
     out.append(do.to(dt) if do is not None else None)
