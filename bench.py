@@ -43,22 +43,40 @@ UNIT = "TFLOP/s"
 TILE = 128
 FLUSH_BYTES = 256 << 20
 
-# DRAM traffic of the dominant kernel (st_attn_bwd_main) per launch, from an ncu capture, valid
-# only while the kernel sources hash to `src`.  Filled in by hand after a capture.
-NCU_TRAFFIC = {
-    # dram read + write, ncu capture at source hash 545233c8f83c2584; the sources changed since
-    # only in host code (the launchers' SM-count helper moved to one place)
-    ("fixed_n12288_l128_c32", "e579f9fa73b1ac01"): 150120448,
+# Per-launch DRAM traffic of the kernels, from the committed ncu table (profiles/), valid while
+# the kernel's sources hash to the value recorded beside it.
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic_by_workload.md")
+KERNEL_SOURCES = {
+    "bwd_kernel": ("bwd.cu", "tiles.cuh", "sm100.cuh", "frames.cuh", "kernels.h"),
+    "fwd_bf16_kernel": ("fwd_bf16.cu", "tiles.cuh", "sm100.cuh", "frames.cuh", "kernels.h"),
 }
 
 
-def kernel_src_hash() -> str:
+def kernel_src_hash(kernel: str = "bwd_kernel") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_factorized_b200", "csrc")
-    for name in ("bwd.cu", "tiles.cuh", "sm100.cuh", "frames.cuh", "kernels.h"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str = "bwd_kernel", path: str = TRAFFIC_TABLE):
+    """DRAM read + write bytes of one step's launches of `kernel` (summed over the passes) from the
+    ncu table, or None when the table has no rows for the workload at the current source hash."""
+    try:
+        with open(path) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    src = kernel_src_hash(kernel)
+    total, found = 0, False
+    for ln in lines:
+        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+        if len(cells) >= 6 and cells[0] == workload and cells[1] == kernel and cells[3] == src:
+            total += int(cells[4]) + int(cells[5])
+            found = True
+    return total if found else None
 
 
 def parse():
@@ -403,8 +421,8 @@ def run_ours(args, rank, world, local):
     peaks = measured_peaks()
     main_ms = statistics.mean(t_main)
     achieved = bwd_flops / (main_ms / 1e3) / 1e12
-    src = kernel_src_hash()
-    tr = NCU_TRAFFIC.get((w.name, src))
+    src = kernel_src_hash("bwd_kernel")
+    tr = recorded_traffic(w.name, "bwd_kernel")
     fwd_bytes, bwd_bytes = step_bytes(w, lay)
     hbm = {"bytes_fwd": fwd_bytes, "bytes_bwd": bwd_bytes,
            "achieved_gbs": (fwd_bytes + bwd_bytes) / (ms / 1e3) / 1e9, "peak_gbs": peaks["hbm_gbs"]}

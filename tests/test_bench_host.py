@@ -121,3 +121,19 @@ def test_cpu_baseline_covers_whole_slabs():
     assert cpu["value"] > 0 and "slabs at full n=512" in cpu["sample"]
     done = int(cpu["sample"].split("oracle fwd+bwd of ")[1].split()[0])
     assert done >= 1
+
+
+def test_traffic_comes_from_the_committed_table_at_the_current_source_hash(tmp_path):
+    """roofline.traffic is read from the ncu table under profiles/ (summed over a workload's
+    passes) only while the kernel's sources hash to the recorded value; otherwise it is None."""
+    src = bench.kernel_src_hash("bwd_kernel")
+    table = tmp_path / "t.md"
+    table.write_text("| workload | kernel | pass | source hash | read | write |\n|---|---|---|---|---|---|\n"
+                     f"| wl_a | bwd_kernel | 1/2 | {src} | 100 | 20 |\n"
+                     f"| wl_a | bwd_kernel | 2/2 | {src} | 7 | 3 |\n"
+                     f"| wl_a | fwd_bf16_kernel | 1/1 | {src} | 999 | 999 |\n"
+                     "| wl_b | bwd_kernel | 1/1 | 0000000000000000 | 5 | 5 |\n")
+    assert bench.recorded_traffic("wl_a", "bwd_kernel", str(table)) == 130
+    assert bench.recorded_traffic("wl_b", "bwd_kernel", str(table)) is None   # stale hash
+    assert bench.recorded_traffic("wl_c", "bwd_kernel", str(table)) is None   # not captured
+    assert bench.recorded_traffic("wl_a", "bwd_kernel", str(tmp_path / "missing.md")) is None
