@@ -282,6 +282,7 @@ CANONICAL_TILES = {
     "strided_merged_n12288_l128": 5104,
     "strided_n65536_l256": 9204,
     "fixed_merged_n12288_l128_c32": 10176,
+    "strided_n12288_l128_d32": 2552,
 }
 
 

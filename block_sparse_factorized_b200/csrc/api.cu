@@ -18,12 +18,14 @@ constexpr size_t FWD_SCHED_BYTES = 256;
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Backward workspace: fp32 dK/dV partial sums of the chunks of split key tiles (one 2 x 128 x 64
-// slot per chunk and batch element) and the item counters of the two passes of the persistent
-// kernel.
+int64_t value_width(const st_desc_t *desc) { return desc->dv == 0 ? desc->d : desc->dv; }
+
+// Backward workspace: fp32 dK/dV partial sums of the chunks of split key tiles (one slot of 128
+// rows x (d + dv) values per chunk and batch element) and the item counters of the two passes of
+// the persistent kernel.
 size_t bwd_partial_bytes(const st_desc_t *desc, const st_layout_t *layout)
 {
-    return static_cast<size_t>(layout->bwd_slots) * desc->batch * 2 * 128 * 64 * sizeof(float);
+    return static_cast<size_t>(layout->bwd_slots) * desc->batch * 128 * (desc->d + value_width(desc)) * sizeof(float);
 }
 size_t bwd_counter_bytes(const st_desc_t *, const st_layout_t *)
 {
@@ -98,73 +100,61 @@ bool make_maps(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH
     return true;
 }
 
-// fp32 [BH, n, 64] maps with 16-column (64-byte, 64-byte swizzle), 32-row boxes: the dQ
-// accumulator as the reduce target of one warp's slice.
-bool make_maps_f32(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col)
+// The swizzle of a box whose rows are `bytes` wide (16: none; 32, 64, 128: the same span), as the
+// backward kernel's per-warp staging writes them.
+CUtensorMapSwizzle swizzle_for(uint32_t bytes)
 {
-    memset(&m, 0, sizeof(m));
-    const cuuint64_t row = 64 * 4, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
-    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    {
-        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
-        const cuuint64_t str[2] = {row, n * row};
-        const cuuint32_t box[3] = {16, 32, 1};
-        if (!encode(&m.nat, base, dt, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
-    }
-    if (col) {
-        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
-        const cuuint64_t str[3] = {l * row, row, n * row};
-        const cuuint32_t rows = static_cast<cuuint32_t>(g.Rt < 32 ? g.Rt : 32);
-        const cuuint32_t slots = static_cast<cuuint32_t>(g.Rt < 32 ? 32 / g.Rt : 1);
-        const cuuint32_t box[4] = {16, rows, slots, 1};
-        if (!encode(&m.col, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
-    }
-    return true;
+    return bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : (bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                       : (bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE));
 }
 
-// bf16 [BH, n, 64] maps with 16-column (32-byte, 32-byte swizzle), 32-row boxes in the natural,
-// grid-column and summary frames: one backward warp's slice of a dK or dV tile.
-bool make_maps_warp16(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum)
+// [BH, n, W] maps with `bx`-column, 32-row boxes in the natural, grid-column and (if sum) summary
+// frames, for one backward warp's slice of rows: the fp32 dQ accumulator as a reduce target
+// (bx = W / 4 fp32), or a warp's slice of a dK or dV tile (bf16).
+bool make_maps_slice(st::FrameMaps &m, const void *base, const st::Geom &g, int64_t BH, bool col, bool sum,
+                     uint32_t W, uint32_t bx, bool f32)
 {
     memset(&m, 0, sizeof(m));
-    const cuuint64_t row = 64 * 2, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
-    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t es = f32 ? 4 : 2, row = W * es, n = static_cast<cuuint64_t>(g.n), l = static_cast<cuuint64_t>(g.l);
+    const CUtensorMapDataType dt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle swz = swizzle_for(static_cast<uint32_t>(bx * es));
     {
-        const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[3] = {W, n, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[2] = {row, n * row};
-        const cuuint32_t box[3] = {16, 32, 1};
-        if (!encode(&m.nat, base, dt, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+        const cuuint32_t box[3] = {bx, 32, 1};
+        if (!encode(&m.nat, base, dt, 3, dims, str, box, swz)) return false;
     }
     if (col) {
-        const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[4] = {W, static_cast<cuuint64_t>(g.R), l, static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[3] = {l * row, row, n * row};
         const cuuint32_t rows = static_cast<cuuint32_t>(g.Rt < 32 ? g.Rt : 32);
         const cuuint32_t slots = static_cast<cuuint32_t>(g.Rt < 32 ? 32 / g.Rt : 1);
-        const cuuint32_t box[4] = {16, rows, slots, 1};
-        if (!encode(&m.col, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+        const cuuint32_t box[4] = {bx, rows, slots, 1};
+        if (!encode(&m.col, base, dt, 4, dims, str, box, swz)) return false;
     }
     if (sum) {
-        const cuuint64_t dims[4] = {64, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
+        const cuuint64_t dims[4] = {W, l, static_cast<cuuint64_t>(g.R), static_cast<cuuint64_t>(BH)};
         const cuuint64_t str[3] = {row, l * row, n * row};
         const cuuint32_t rows = static_cast<cuuint32_t>(g.c < 32 ? g.c : 32);
         const cuuint32_t runs = static_cast<cuuint32_t>(g.c < 32 ? 32 / g.c : 1);
-        const cuuint32_t box[4] = {16, rows, runs, 1};
-        if (!encode(&m.sum, base, dt, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+        const cuuint32_t box[4] = {bx, rows, runs, 1};
+        if (!encode(&m.sum, base, dt, 4, dims, str, box, swz)) return false;
     }
     return true;
 }
 
-// The dQ output in the natural frame with a 16-column, 32-row box: one warp's slice of a query
-// tile whose dQ the backward kernel stores directly (fp32: 64-byte swizzle, as the accumulator's
-// reduce map; bf16: 32-byte rows, 32-byte swizzle).
-bool make_map_dq_direct(CUtensorMap *m, const void *base, const st::Geom &g, int64_t BH, bool f32)
+// The dQ output [BH, n, W] in the natural frame with a W / 4-column, 32-row box: one warp's slice
+// of a query tile whose dQ the backward kernel stores directly (fp32 or bf16, swizzled as the
+// kernel stages it).
+bool make_map_dq_direct(CUtensorMap *m, const void *base, const st::Geom &g, int64_t BH, bool f32, uint32_t W)
 {
-    const cuuint64_t row = 64 * (f32 ? 4 : 2), n = static_cast<cuuint64_t>(g.n);
-    const cuuint64_t dims[3] = {64, n, static_cast<cuuint64_t>(BH)};
+    const cuuint64_t es = f32 ? 4 : 2, row = W * es, n = static_cast<cuuint64_t>(g.n);
+    const cuuint64_t dims[3] = {W, n, static_cast<cuuint64_t>(BH)};
     const cuuint64_t str[2] = {row, n * row};
-    const cuuint32_t box[3] = {16, 32, 1};
+    const cuuint32_t box[3] = {W / 4, 32, 1};
     return encode(m, base, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dims, str,
-                  box, f32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+                  box, swizzle_for(static_cast<uint32_t>(W / 4 * es)));
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -184,15 +174,14 @@ Frames frames_used(const st_layout &L)
     return f;
 }
 
-int64_t value_width(const st_desc_t *desc) { return desc->dv == 0 ? desc->d : desc->dv; }
-
-// Row widths the kernels are built for.  The bf16 forward: (query-key, value) = (32, 32),
-// (64, 64), (128, 128), (64, 128).  Everything else: 64 and 64.
+// Row widths the kernels are built for (query-key, value).  bf16 forward: (32, 32), (64, 64),
+// (128, 128), (64, 128); bf16 backward: (32, 32), (64, 64), (64, 128); fp32 I/O: (64, 64).
 bool widths_supported(const st_desc_t *desc, bool fwd = false)
 {
     const int64_t dv = value_width(desc);
-    if (fwd && desc->dtype == ST_BF16 && desc->d <= 128 && dv <= 128)
-        return st::fwd_bf16_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv));
+    if (desc->dtype == ST_BF16 && desc->d <= 128 && dv <= 128)
+        return fwd ? st::fwd_bf16_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv))
+                   : st::bwd_widths_supported(static_cast<int>(desc->d), static_cast<int>(dv));
     return desc->d == 64 && dv == 64;
 }
 
@@ -256,7 +245,7 @@ size_t st_attn_bwd_workspace_bytes(const st_desc_t *desc, const st_layout_t *lay
 {
     if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
-    const size_t dq = rows * 64 * sizeof(float);
+    const size_t dq = rows * desc->d * sizeof(float);
     const size_t dl = rows * sizeof(float);
     const size_t base = round256(dq) + round256(dl) + round256(bwd_partial_bytes(desc, layout)) +
                         round256(bwd_counter_bytes(desc, layout));
@@ -337,7 +326,7 @@ st_status_t bwd_workspace(const st_desc_t *desc, const st_layout_t *layout, void
     const size_t rows = static_cast<size_t>(desc->batch) * desc->heads * desc->n;
     char *w = static_cast<char *>(workspace);
     ws.dq_acc = reinterpret_cast<float *>(w);
-    w += round256(rows * 64 * sizeof(float));
+    w += round256(rows * desc->d * sizeof(float));
     ws.delta = reinterpret_cast<float *>(w);
     w += round256(rows * sizeof(float));
     ws.partials = reinterpret_cast<float *>(w);
@@ -381,7 +370,10 @@ st_status_t st_attn_bwd_prepare(const void *o, const void *dO, const st_layout_t
     pre.bh = desc->batch * desc->heads;
     pre.n = static_cast<int32_t>(desc->n);
     pre.heads = static_cast<int32_t>(desc->heads);
-    return st::launch_bwd_pre(pre, f32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+    return st::launch_bwd_pre(pre, f32, static_cast<int>(desc->d), static_cast<int>(value_width(desc)), stream) ==
+                   cudaSuccess
+               ? ST_OK
+               : ST_ERR_CUDA;
 }
 
 st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const float *lse,
@@ -417,20 +409,21 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
         p.dk_f32 = static_cast<float *>(dk);
         p.dv_f32 = static_cast<float *>(dv);
     }
-    if (!make_map_dq_direct(&p.dq_direct, dq, L.geom, BH, f32)) return ST_ERR_CUDA;
-    if (!make_maps_f32(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol)) return ST_ERR_CUDA;
-    if (!f32 && (!make_maps_warp16(p.dk_w, dk, L.geom, BH, f.kcol, f.ksum) ||
-                 !make_maps_warp16(p.dv_w, dv, L.geom, BH, f.kcol, f.ksum)))
+    const uint32_t dqk = static_cast<uint32_t>(desc->d), dvw = static_cast<uint32_t>(value_width(desc));
+    if (!make_map_dq_direct(&p.dq_direct, dq, L.geom, BH, f32, dqk)) return ST_ERR_CUDA;
+    if (!make_maps_slice(p.dq_red, ws.dq_acc, L.geom, BH, f.qcol, false, dqk, dqk / 4, true)) return ST_ERR_CUDA;
+    if (!f32 && (!make_maps_slice(p.dk_w, dk, L.geom, BH, f.kcol, f.ksum, dqk, dqk / 4, false) ||
+                 !make_maps_slice(p.dv_w, dv, L.geom, BH, f.kcol, f.ksum, dvw, dvw / 4, false)))
         return ST_ERR_CUDA;
-    if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false) ||
-        !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum))
+    if (!make_maps(p.q, qb, L.geom, BH, f.qcol, false, dqk) || !make_maps(p.dout, dob, L.geom, BH, f.qcol, false, dvw) ||
+        !make_maps(p.k, kb, L.geom, BH, f.kcol, f.ksum, dqk) || !make_maps(p.v, vb, L.geom, BH, f.kcol, f.ksum, dvw))
         return ST_ERR_CUDA;
     p.parts = L.d_parts;
     p.batch = static_cast<int32_t>(desc->batch);
     p.heads = static_cast<int32_t>(desc->heads);
     p.g = L.geom;
-    p.scale_log2 = LOG2E / 8.0f;
-    p.ds_scale = 1.0f / 8.0f;
+    p.scale_log2 = LOG2E / sqrtf(static_cast<float>(dqk));  // log2(e) / sqrt(d)
+    p.ds_scale = 1.0f / sqrtf(static_cast<float>(dqk));
     p.lse = lse;
     p.delta = ws.delta;
     p.dq_acc = ws.dq_acc;
@@ -444,7 +437,8 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
         p.items = L.d_bwd[pass];
         p.nitems = static_cast<int32_t>(L.bwd_items[pass].size());
         p.sched = ws.counters + pass;
-        if (st::launch_bwd(p, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
+        if (st::launch_bwd(p, f32, static_cast<int>(dqk), static_cast<int>(dvw), stream) != cudaSuccess)
+            return ST_ERR_CUDA;
         // split key tiles of this pass: the next pass (a merge) reads their dK/dV
         st::SplitFinishParams sf;
         memset(&sf, 0, sizeof(sf));
@@ -461,7 +455,8 @@ st_status_t st_attn_bwd_main(const void *q, const void *k, const void *v, const 
             sf.dk_f32 = static_cast<float *>(dk);
             sf.dv_f32 = static_cast<float *>(dv);
         }
-        if (st::launch_split_finish(sf, f32, stream) != cudaSuccess) return ST_ERR_CUDA;
+        if (st::launch_split_finish(sf, f32, static_cast<int>(dqk), static_cast<int>(dvw), stream) != cudaSuccess)
+            return ST_ERR_CUDA;
     }
     return ST_OK;
 }
@@ -485,7 +480,9 @@ st_status_t st_attn_bwd_finish(const st_layout_t *layout, void *dq, void *worksp
     cv.batch = static_cast<int32_t>(desc->batch);
     cv.n = static_cast<int32_t>(desc->n);
     cv.heads = static_cast<int32_t>(desc->heads);
-    return st::launch_dq_convert(cv, desc->dtype == ST_FP32, stream) == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+    return st::launch_dq_convert(cv, desc->dtype == ST_FP32, static_cast<int>(desc->d), stream) == cudaSuccess
+               ? ST_OK
+               : ST_ERR_CUDA;
 }
 
 st_status_t st_attn_bwd(const void *q, const void *k, const void *v, const void *o,

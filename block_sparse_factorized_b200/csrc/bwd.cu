@@ -29,36 +29,53 @@
 //               two TMA stores (bf16), written row by row (fp32), or stored as the fp32 partial
 //               of a split key tile.
 // A merge part (second pass of a merged head) adds the dK/dV the first pass wrote.
+#include <type_traits>
+
 #include "tiles.cuh"
 
 namespace st {
 namespace {
 
-constexpr uint32_t TB = TILE_BYTES;
-constexpr int NST = 2;                             // Q/dO ring depth
+constexpr uint32_t TB = TILE_BYTES;              // a 128 x 128 bf16 operand half (P, dS): 16 KB
 constexpr int NSCHED = 4;                          // claimed-item ring depth
-constexpr int KVS = 2;                             // K/V slots (items in flight)
-constexpr uint32_t OFF_K = 0;                      // KVS slots
-constexpr uint32_t OFF_V = OFF_K + KVS * TB;       // KVS slots
-constexpr uint32_t OFF_Q = OFF_V + KVS * TB;       // NST tiles
-constexpr uint32_t OFF_DO = OFF_Q + NST * TB;      // NST tiles
-constexpr uint32_t OFF_P = OFF_DO + NST * TB;      // 2 halves
-constexpr uint32_t OFF_DS = OFF_P + 2 * TB;        // 2 halves
-constexpr uint32_t OFF_DQ = OFF_DS + 2 * TB;       // dQ staging: 2 x (128 rows x 32 fp32)
-constexpr uint32_t OFF_BAR = OFF_DQ + 2 * TB;
-constexpr uint32_t OFF_ITEMS = OFF_BAR + 256;      // the claimed items' fields, NSCHED entries
-constexpr uint32_t SMEM_BYTES = OFF_ITEMS + NSCHED * 96;
 constexpr int NWG = 4;                             // softmax warpgroups
 constexpr int NSM = 128 * NWG;                     // softmax threads
 constexpr int THREADS = 64 + NSM;
 constexpr int CW = 128 / NWG;                      // score columns per warpgroup (32)
-constexpr int OW = 64 / NWG;                       // dQ / dK / dV columns per warpgroup (16)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 320, COL_DQ = 384;
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256;
+constexpr int MAX_STAGES = 2;                      // ring depths are at most this
+
+// Query-key rows of width DQK, value rows of width DV.
+template <int DQK, int DV>
+struct BCfg {
+    static constexpr uint32_t QB = Tile<DQK>::BYTES, VB = Tile<DV>::BYTES;  // Q or K tile, V or dO tile
+    // ring depths: 128-wide value rows fit shared memory only with single buffers
+    static constexpr int KVS = DV > 64 ? 1 : 2;    // K/V slots (items in flight)
+    static constexpr int NST = DV > 64 ? 1 : 2;    // Q/dO ring depth
+    static constexpr int OWQ = DQK / NWG;          // dQ / dK columns per warpgroup
+    static constexpr int OWV = DV / NWG;           // dV columns per warpgroup
+    // per-warp staging: the dQ slice (32 rows x OWQ fp32), or the dK and dV slices (bf16)
+    static constexpr uint32_t STG_DQ = 32 * OWQ * 4, STG_DK = 32 * OWQ * 2, STG_DV = 32 * OWV * 2;
+    static constexpr uint32_t STG = STG_DQ > STG_DK + STG_DV ? STG_DQ : STG_DK + STG_DV;
+    static constexpr uint32_t OFF_K = 0;                       // KVS slots
+    static constexpr uint32_t OFF_V = OFF_K + KVS * QB;        // KVS slots
+    static constexpr uint32_t OFF_Q = OFF_V + KVS * VB;        // NST tiles
+    static constexpr uint32_t OFF_DO = OFF_Q + NST * QB;       // NST tiles
+    static constexpr uint32_t OFF_P = OFF_DO + NST * VB;       // 2 halves
+    static constexpr uint32_t OFF_DS = OFF_P + 2 * TB;         // 2 halves
+    static constexpr uint32_t OFF_DQ = OFF_DS + 2 * TB;        // staging, NSM / 32 warps
+    static constexpr uint32_t OFF_BAR = OFF_DQ + (NSM / 32) * ((STG + 1023) & ~1023u);
+    static constexpr uint32_t OFF_ITEMS = OFF_BAR + 256;       // the claimed items' fields
+    static constexpr uint32_t SMEM_BYTES = OFF_ITEMS + NSCHED * 96;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static constexpr uint32_t COL_DK = COL_DV + DV, COL_DQ = COL_DK + DQK;
+    static_assert(COL_DQ + DQK <= TMEM_COLS, "tensor memory");
+};
 
 struct Bars {
-    uint64_t kv_full[KVS], kv_empty[KVS];
-    uint64_t qdo_full[NST], qdo_empty[NST];
+    uint64_t kv_full[MAX_STAGES], kv_empty[MAX_STAGES];
+    uint64_t qdo_full[MAX_STAGES], qdo_empty[MAX_STAGES];
     uint64_t s_full, dp_full, p_ready, ds_ready, dq_full, dq_empty;
     uint64_t acc_free;             // the epilogue has read dK and dV of the item from TMEM
     uint64_t mma_idle;             // every MMA this CTA issued has completed (before teardown)
@@ -107,10 +124,18 @@ __device__ __forceinline__ void done_item(Bars *bars, int32_t j, bool warp_wide)
     if (!warp_wide || (threadIdx.x & 31) == 0) mbar_arrive(&bars->sched_empty[j % NSCHED]);
 }
 
-// F32: fp32 I/O -- dK and dV are written in fp32 (the MMAs run on bf16 copies).
-template <bool F32>
+// F32: fp32 I/O -- dK and dV are written in fp32 (the MMAs run on bf16 copies; query-key and
+// value rows of 64).  DQK, DV: the widths of the query-key and value rows.
+template <bool F32, int DQK, int DV>
 __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p)
 {
+    using C = BCfg<DQK, DV>;
+    constexpr int KVS = C::KVS, NST = C::NST, OWQ = C::OWQ, OWV = C::OWV;
+    constexpr uint32_t QB = C::QB, VB = C::VB, OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_Q = C::OFF_Q,
+                       OFF_DO = C::OFF_DO, OFF_P = C::OFF_P, OFF_DS = C::OFF_DS, OFF_DQ = C::OFF_DQ,
+                       OFF_BAR = C::OFF_BAR, OFF_ITEMS = C::OFF_ITEMS, COL_DK = C::COL_DK,
+                       COL_DQ = C::COL_DQ;
+    static_assert(!F32 || (DQK == 64 && DV == 64), "fp32 I/O has rows of 64");
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BAR);
@@ -180,9 +205,11 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                 const Item it = *slot;
                 const int ks = I % KVS;
                 if (I >= KVS && !mbar_wait(&bars->kv_empty[ks], ((I / KVS) - 1) & 1, abort, p.err)) break;
-                mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * TB);
-                load_tile(p.k, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_K + ks * TB, &bars->kv_full[ks]);
-                load_tile(p.v, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_V + ks * TB, &bars->kv_full[ks]);
+                mbar_arrive_expect_tx(&bars->kv_full[ks], QB + VB);
+                load_tile_w<DQK>(p.k, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_K + ks * QB,
+                                 &bars->kv_full[ks]);
+                load_tile_w<DV>(p.v, it.part.kframe, p.g, it.part.o, it.w.tile, it.bh, smem + OFF_V + ks * VB,
+                                &bars->kv_full[ks]);
                 ++I;
                 for (int32_t jj = 0; jj < it.nq; ++jj, ++J) {
                     const int qs = J % NST;
@@ -190,11 +217,11 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                         fail = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars->qdo_full[qs], 2 * TB);
-                    load_tile(p.q, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh, smem + OFF_Q + qs * TB,
-                              &bars->qdo_full[qs]);
-                    load_tile(p.dout, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh,
-                              smem + OFF_DO + qs * TB, &bars->qdo_full[qs]);
+                    mbar_arrive_expect_tx(&bars->qdo_full[qs], QB + VB);
+                    load_tile_w<DQK>(p.q, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh,
+                                     smem + OFF_Q + qs * QB, &bars->qdo_full[qs]);
+                    load_tile_w<DV>(p.dout, it.part.qframe, p.g, it.part.o, it.w.begin + jj, it.bh,
+                                    smem + OFF_DO + qs * VB, &bars->qdo_full[qs]);
                 }
             }
             if (*abort) {  // drain the copies still in flight before the CTA leaves
@@ -209,28 +236,31 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         // ---------------- MMA issuer ----------------
         if (lane == 0 && run) {
             constexpr uint32_t id_nn = idesc_bf16(128, 128, false, false);  // S, dP
-            constexpr uint32_t id_tt = idesc_bf16(128, 64, true, true);     // dV, dK
-            constexpr uint32_t id_kt = idesc_bf16(128, 64, false, true);    // dQ
+            constexpr uint32_t id_tv = idesc_bf16(128, DV, true, true);     // dV
+            constexpr uint32_t id_tk = idesc_bf16(128, DQK, true, true);    // dK
+            constexpr uint32_t id_kt = idesc_bf16(128, DQK, false, true);   // dQ
             const uint32_t sP = smem_u32(smem + OFF_P), sDS = smem_u32(smem + OFF_DS);
-            auto sQ = [&](int32_t t) { return smem_u32(smem + OFF_Q + (t % NST) * TB); };
-            auto sDO = [&](int32_t t) { return smem_u32(smem + OFF_DO + (t % NST) * TB); };
+            auto sQ = [&](int32_t t) { return smem_u32(smem + OFF_Q + (t % NST) * QB); };
+            auto sDO = [&](int32_t t) { return smem_u32(smem + OFF_DO + (t % NST) * VB); };
+            auto sKs = [&](int32_t slot) { return smem_u32(smem + OFF_K + slot * QB); };
+            auto sVs = [&](int32_t slot) { return smem_u32(smem + OFF_V + slot * VB); };
             // Per query tile t the tensor core runs, in order:
             //   dV += P_t^T dO_t | S_{t+1} | dQ_t = dS_t K, dK += dS_t^T Q_t | dP_{t+1}
             // so that it computes dV_t and S_{t+1} while the softmax warps build dS_t, and dK_t,
             // dQ_t, dP_{t+1} while they drain dQ_t and build P_{t+1}.  An item's first S and dP
             // follow the previous item's last dQ.
-            auto issue_s = [&](uint32_t q, uint32_t k) {  // S = Q K^T (both K-major over d)
+            auto issue_s = [&](uint32_t q, uint32_t k) {  // S = Q K^T (both K-major over DQK)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + COL_S, desc_sw128(q + 32 * kk, 16, 1024),
-                                desc_sw128(k + 32 * kk, 16, 1024), id_nn, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < DQK / 16; ++kk)
+                    mma_bf16_ss(tbase + COL_S, Tile<DQK>::kmajor(q, kk), Tile<DQK>::kmajor(k, kk), id_nn,
+                                kk > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full);
             };
-            auto issue_dp = [&](uint32_t o, uint32_t v) {  // dP = dO V^T
+            auto issue_dp = [&](uint32_t o, uint32_t v) {  // dP = dO V^T (both K-major over DV)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + COL_DP, desc_sw128(o + 32 * kk, 16, 1024),
-                                desc_sw128(v + 32 * kk, 16, 1024), id_nn, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < DV / 16; ++kk)
+                    mma_bf16_ss(tbase + COL_DP, Tile<DV>::kmajor(o, kk), Tile<DV>::kmajor(v, kk), id_nn,
+                                kk > 0 ? 1u : 0u);
                 mma_commit(&bars->dp_full);
             };
             // One flat loop over the query tiles of all items this CTA claims: the tile after the
@@ -247,8 +277,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                           mbar_wait(&bars->qdo_full[0], 0, abort, p.err);
                 if (ok) {
                     tc_fence_after();
-                    issue_s(sQ(0), smem_u32(smem + OFF_K));
-                    issue_dp(sDO(0), smem_u32(smem + OFF_V));
+                    issue_s(sQ(0), sKs(0));
+                    issue_dp(sDO(0), sVs(0));
                 }
                 while (ok) {
                     const int32_t t = J;
@@ -267,42 +297,49 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     if (jj == 0 && I > 0 && !mbar_wait(&bars->acc_free, (I - 1) & 1, abort, p.err)) break;
                     tc_fence_after();
                     // dV += P^T dO: A = P^T MN-major (two 64-key atoms 16 KB apart), B = dO
-                    // MN-major; 16 queries (2048 bytes) per step
+                    // MN-major; 16 queries per step
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + kk * 2048, TB, 1024),
-                                    desc_sw128(sDO(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
-                    if (has_next) {  // S of the next tile: the softmax warps are done reading S_t
+                        mma_bf16_ss(tbase + COL_DV, desc_sw128(sP + kk * 2048, TB, 1024), Tile<DV>::mnmajor(sDO(t), kk),
+                                    id_tv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    // S of the next tile: the softmax warps are done reading S_t.  With single
+                    // buffers (a one-stage Q/dO ring, or one K/V slot at an item's last tile) the
+                    // next tile's Q or K takes the slot of this tile's, so its S follows dK below.
+                    const bool late_s = NST == 1 || (last && KVS == 1);
+                    auto next_s = [&]() {
                         if (!mbar_wait(&bars->qdo_full[(t + 1) % NST], ((t + 1) / NST) & 1, abort, p.err) ||
                             (last && !mbar_wait(&bars->kv_full[nks], ((I + 1) / KVS) & 1, abort, p.err)))
-                            break;
+                            return false;
                         tc_fence_after();
-                        issue_s(sQ(t + 1), smem_u32(smem + OFF_K + nks * TB));
-                    }
+                        issue_s(sQ(t + 1), sKs(nks));
+                        return true;
+                    };
+                    if (has_next && !late_s && !next_s()) break;
                     if (!mbar_wait(&bars->ds_ready, t & 1, abort, p.err) ||
                         (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort, p.err)))
                         break;
                     tc_fence_after();
-                    const uint32_t sK = smem_u32(smem + OFF_K + ks * TB);
+                    const uint32_t sK = sKs(ks);
                     // dQ = dS K (A = dS K-major, two 64-key halves; B = K MN-major), signalled at once
                     // so that the drain can start, then dK += dS^T Q (as dV); on an item's last tile
                     // dq_full waits for dK too, since the epilogue reads it
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ss(tbase + COL_DQ, desc_sw128(sDS + (kk >> 2) * TB + (kk & 3) * 32, 16, 1024),
-                                    desc_sw128(sK + kk * 2048, TB, 1024), id_kt, kk > 0 ? 1u : 0u);
+                                    Tile<DQK>::mnmajor(sK, kk), id_kt, kk > 0 ? 1u : 0u);
                     if (!last) mma_commit(&bars->dq_full);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + kk * 2048, TB, 1024),
-                                    desc_sw128(sQ(t) + kk * 2048, TB, 1024), id_tt, (jj > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ss(tbase + COL_DK, desc_sw128(sDS + kk * 2048, TB, 1024), Tile<DQK>::mnmajor(sQ(t), kk),
+                                    id_tk, (jj > 0 || kk > 0) ? 1u : 0u);
                     if (last) mma_commit(&bars->dq_full);  // also: dK, dV of the item complete
                     mma_commit(&bars->qdo_empty[t % NST]);
                     if (last) {
                         mma_commit(&bars->kv_empty[ks]);  // K and V of this item are no longer read
                         done_item(bars, j, false);
                     }
-                    if (has_next) issue_dp(sDO(t + 1), smem_u32(smem + OFF_V + nks * TB));  // dP_t consumed
+                    if (has_next && late_s && !next_s()) break;
+                    if (has_next) issue_dp(sDO(t + 1), sVs(nks));  // dP_t consumed
                     ++J;
                     if (!has_next) break;
                     if (last) {
@@ -328,12 +365,13 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
         const int row = q4 * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
         const uint32_t tS = tbase + COL_S + lane_off + CW * g, tDP = tbase + COL_DP + lane_off + CW * g;
-        const uint32_t tDQ = tbase + COL_DQ + lane_off + OW * g;
+        const uint32_t tDQ = tbase + COL_DQ + lane_off + OWQ * g;
         // P and dS live in two 128 x 64 swizzled halves; this warpgroup's 32 columns are four
         // 16-byte chunks of half g/2
         const uint32_t sPg = smem_u32(smem + OFF_P) + (g >> 1) * TB, sDSg = smem_u32(smem + OFF_DS) + (g >> 1) * TB;
         const uint32_t chunk0 = (g & 1) * 4;
-        const uint32_t warp_slot = (g * 4 + q4) * 2048;     // this warp's dQ staging (32 x 64 B)
+        // this warp's staging: its dQ slice (32 rows x OWQ fp32) or its dK and dV slices (bf16)
+        const uint32_t warp_slot = (g * 4 + q4) * ((C::STG + 1023) & ~1023u);
         const uint32_t sDQw = smem_u32(smem + OFF_DQ) + warp_slot;
         const float sc = p.scale_log2, dsc = p.ds_scale;
         bool ok = run;
@@ -422,38 +460,38 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
             tc_fence_before();
             mbar_arrive(&bars->ds_ready);
         };
-        auto drain = [&](int32_t t, int32_t jj) {  // dQ_t columns OW g.. : TMEM -> SMEM -> TMA reduce-add
+        auto drain = [&](int32_t t, int32_t jj) {  // dQ_t columns OWQ g.. : TMEM -> SMEM -> TMA reduce-add
             if (!wait_all(&bars->dq_full, t & 1)) return;
-            uint32_t dq[16];
-            tmem_ld16(tDQ, dq);
+            uint32_t dq[OWQ];
+            tmem_ld_n<OWQ>(tDQ, dq);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
-            // per-warp staging (32 rows x 64 bytes, 64-byte swizzle): no cross-warp barrier
+            // per-warp staging (32 rows, swizzled as the TMA map of the slice): no cross-warp barrier
             if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce / store has read it
             __syncwarp();
             const bool direct = cur->part.dq_direct != 0;  // the only contribution to these rows
-            if (!F32 && direct) {  // bf16 dQ itself: 32 rows x 32 bytes, 32-byte swizzle
+            if (!F32 && direct) {  // bf16 dQ itself: 32 rows x 2 OWQ bytes
 #pragma unroll
-                for (int q = 0; q < 2; ++q)
-                    st_shared_v4(sDQw + sw32_off(lane, q),
+                for (int q = 0; q < OWQ / 8; ++q)
+                    st_shared_v4(sDQw + swz_off<2 * OWQ>(lane, q),
                                  pack_bf16(__uint_as_float(dq[8 * q]), __uint_as_float(dq[8 * q + 1])),
                                  pack_bf16(__uint_as_float(dq[8 * q + 2]), __uint_as_float(dq[8 * q + 3])),
                                  pack_bf16(__uint_as_float(dq[8 * q + 4]), __uint_as_float(dq[8 * q + 5])),
                                  pack_bf16(__uint_as_float(dq[8 * q + 6]), __uint_as_float(dq[8 * q + 7])));
-            } else {
+            } else {  // fp32: 32 rows x 4 OWQ bytes
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    st_shared_v4(sDQw + sw64_off(lane, q), dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
+                for (int q = 0; q < OWQ / 4; ++q)
+                    st_shared_v4(sDQw + swz_off<4 * OWQ>(lane, q), dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 if (direct)  // a natural-frame query part: a plain TMA store of the slice
-                    tma_store_3d(&p.dq_direct, smem + OFF_DQ + warp_slot, OW * g,
+                    tma_store_3d(&p.dq_direct, smem + OFF_DQ + warp_slot, OWQ * g,
                                  (cur->w.begin + jj) * TILE + 32 * q4, cur->bh);
                 else
-                    reduce_warp_f32(p.dq_red, cur->part.qframe, p.g, cur->w.begin + jj, cur->bh, OW * g, q4,
+                    reduce_warp_f32(p.dq_red, cur->part.qframe, p.g, cur->w.begin + jj, cur->bh, OWQ * g, q4,
                                     smem + OFF_DQ + warp_slot);
                 bulk_commit();
             }
@@ -494,116 +532,97 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
                     ++jj;
                     continue;
                 }
-                // ------- dK, dV of the item: one key row per thread, warpgroup g owns columns OW g.. -------
+                // ------- dK, dV of the item: one key row per thread, warpgroup g owns dK columns
+                // OWQ g.. and dV columns OWV g.. -------
                 // (the last drain waited for dq_full of the item's last tile, whose commit covers
                 // every dK and dV product of the item).  The next item's P_0 is already built; its
                 // first dV product waits for acc_free, arrived below.
                 const int32_t pos = frame_pos(p.g, cur->part.kframe, cur->part.o, cur->w.tile, row);
-                // output of one row slice: add the first pass's values for a merge part (read by this
-                // same thread), round, store
-                auto emit = [&](int which, float (&a)[OW]) {
-                    const size_t off = (head_base + pos) * 64 + OW * g;
-                    if (F32) {
-                        float *of = (which == 0 ? p.dk_f32 : p.dv_f32) + off;
-                        if (cur->part.merge) {
-                            const float4 *src = reinterpret_cast<const float4 *>(of);
-#pragma unroll
-                            for (int q = 0; q < OW / 4; ++q) {
-                                const float4 x = src[q];
-                                a[4 * q] += x.x;
-                                a[4 * q + 1] += x.y;
-                                a[4 * q + 2] += x.z;
-                                a[4 * q + 3] += x.w;
-                            }
-                        }
-                        float4 *d4 = reinterpret_cast<float4 *>(of);
-#pragma unroll
-                        for (int q = 0; q < OW / 4; ++q) d4[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-                    } else {
-                        uint4 *d4 = reinterpret_cast<uint4 *>((which == 0 ? p.dk_out : p.dv_out) + off);
-                        if (cur->part.merge) {
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const uint4 x = d4[q];
-                                const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    a[8 * q + 2 * e] += bf16_lo(xx[e]);
-                                    a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
-                                }
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < 2; ++q)
-                            d4[q] = make_uint4(pack_bf16(a[8 * q], a[8 * q + 1]), pack_bf16(a[8 * q + 2], a[8 * q + 3]),
-                                               pack_bf16(a[8 * q + 4], a[8 * q + 5]), pack_bf16(a[8 * q + 6], a[8 * q + 7]));
-                    }
-                };
                 // Chunk of a split key tile: store the fp32 partial in this chunk's slot (a pass after
                 // the kernel adds the chunks' slots in chunk order and writes dK and dV), in thread
-                // order: uint4 ((which * 4 + q) * 4 + g) * 128 + row, so that each warp store is 512
-                // contiguous bytes.  bf16 output: each warp stages its 32 rows x 16 columns of dK and
-                // dV in its own dQ staging slot and writes them with two TMA stores (no cross-warp
-                // barrier; the warp's next dQ drain waits for their reads as for a reduce).
-                constexpr size_t SLOT = 2 * 128 * 64;
+                // order: dK's 16-byte group q of slice g of row r at uint4 (q * 4 + g) * 128 + r, dV's
+                // after all of dK's (DQK * 32 uint4 further), so that each warp store is 512
+                // contiguous bytes.  bf16 output: each warp stages its 32 rows of dK and dV in its
+                // own staging slot and writes them with two TMA stores (no cross-warp barrier; the
+                // warp's next dQ drain waits for their reads as for a reduce).
+                constexpr size_t SLOT = static_cast<size_t>(128) * (DQK + DV);
                 const bool split = cur->w.slot >= 0;
                 const bool staged = !F32 && !split;
                 if (staged) {
                     if (lane == 0) bulk_wait_read_all();  // this warp's last reduce has read the slot
                     __syncwarp();
                 }
-#pragma unroll
-                for (int which = 0; which < 2; ++which) {
-                    uint32_t a16[OW];
-                    tmem_ld16(tbase + (which == 0 ? COL_DK : COL_DV) + lane_off + OW * g, a16);
+                // one of the two outputs: W columns from TMEM column col, partial-slot offset part0
+                // (uint4), first-pass values and output rows of `width` elements at out / out_f32,
+                // staging at stg
+                auto emit = [&](auto Wc, uint32_t col, size_t part0, uint16_t *out, float *out_f32, int32_t width,
+                                uint32_t stg) {
+                    constexpr int W = decltype(Wc)::value;
+                    uint32_t a16[W];
+                    tmem_ld_n<W>(tbase + col + lane_off + W * g, a16);
                     tmem_wait_ld();
-                    if (*abort != 0) continue;
+                    if (*abort != 0) return;
                     if (split) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.partials + (static_cast<size_t>(cur->w.slot) * p.batch + cur->b) * SLOT);
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.partials + (static_cast<size_t>(cur->w.slot) * p.batch + cur->b) * SLOT) + part0;
 #pragma unroll
-                        for (int q = 0; q < OW / 4; ++q)
-                            dst[((which * 4 + q) * 4 + g) * 128 + row] = make_uint4(a16[4 * q], a16[4 * q + 1], a16[4 * q + 2], a16[4 * q + 3]);
-                    } else {
-                        float a[OW];
+                        for (int q = 0; q < W / 4; ++q)
+                            dst[(q * 4 + g) * 128 + row] = make_uint4(a16[4 * q], a16[4 * q + 1], a16[4 * q + 2], a16[4 * q + 3]);
+                        return;
+                    }
+                    float a[W];
 #pragma unroll
-                        for (int e = 0; e < OW; ++e) a[e] = __uint_as_float(a16[e]);
-                        if (F32) {
-                            if (pos >= 0) emit(which, a);
-                        } else {
-                            if (cur->part.merge && pos >= 0) {  // add the first pass's values
-                                const uint4 *src = reinterpret_cast<const uint4 *>((which == 0 ? p.dk_out : p.dv_out) +
-                                                                                   (head_base + pos) * 64 + OW * g);
+                    for (int e = 0; e < W; ++e) a[e] = __uint_as_float(a16[e]);
+                    if (pos < 0) return;  // frame padding
+                    const size_t off = (head_base + pos) * width + W * g;
+                    if (F32) {  // rows of the fp32 output, the first pass's values added by this thread
+                        float4 *d4 = reinterpret_cast<float4 *>(out_f32 + off);
 #pragma unroll
-                                for (int q = 0; q < 2; ++q) {
-                                    const uint4 x = src[q];
-                                    const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        a[8 * q + 2 * e] += bf16_lo(xx[e]);
-                                        a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
-                                    }
-                                }
+                        for (int q = 0; q < W / 4; ++q) {
+                            float4 v = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                            if (cur->part.merge) {
+                                const float4 x = d4[q];
+                                v.x += x.x;
+                                v.y += x.y;
+                                v.z += x.z;
+                                v.w += x.w;
                             }
-                            // this warp's slice: 32 rows x 32 bytes, 32-byte swizzle (dK, then dV)
-                            const uint32_t dst = sDQw + which * 1024;
+                            d4[q] = v;
+                        }
+                        return;
+                    }
+                    if (cur->part.merge) {  // add the first pass's values
+                        const uint4 *src = reinterpret_cast<const uint4 *>(out + off);
 #pragma unroll
-                            for (int q = 0; q < 2; ++q)
-                                st_shared_v4(dst + sw32_off(lane, q), pack_bf16(a[8 * q], a[8 * q + 1]),
-                                             pack_bf16(a[8 * q + 2], a[8 * q + 3]), pack_bf16(a[8 * q + 4], a[8 * q + 5]),
-                                             pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+                        for (int q = 0; q < W / 8; ++q) {
+                            const uint4 x = src[q];
+                            const uint32_t xx[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                a[8 * q + 2 * e] += bf16_lo(xx[e]);
+                                a[8 * q + 2 * e + 1] += bf16_hi(xx[e]);
+                            }
                         }
                     }
-                }
+                    // this warp's slice: 32 rows x 2 W bytes, swizzled as the slice's TMA map
+#pragma unroll
+                    for (int q = 0; q < W / 8; ++q)
+                        st_shared_v4(stg + swz_off<2 * W>(lane, q), pack_bf16(a[8 * q], a[8 * q + 1]),
+                                     pack_bf16(a[8 * q + 2], a[8 * q + 3]), pack_bf16(a[8 * q + 4], a[8 * q + 5]),
+                                     pack_bf16(a[8 * q + 6], a[8 * q + 7]));
+                };
+                emit(std::integral_constant<int, OWQ>(), COL_DK, 0, p.dk_out, p.dk_f32, DQK, sDQw);
+                emit(std::integral_constant<int, OWV>(), COL_DV, static_cast<size_t>(DQK) * 32, p.dv_out, p.dv_f32, DV,
+                     sDQw + C::STG_DK);
                 tc_fence_before();
                 mbar_arrive(&bars->acc_free);  // the next item's first dV, dK may overwrite them
                 if (staged) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        store_warp_slice(p.dk_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OW * g, q4,
+                        store_warp_slice(p.dk_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OWQ * g, q4,
                                          smem + OFF_DQ + warp_slot);
-                        store_warp_slice(p.dv_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OW * g, q4,
-                                         smem + OFF_DQ + warp_slot + 1024);
+                        store_warp_slice(p.dv_w, cur->part.kframe, p.g, cur->part.o, cur->w.tile, cur->bh, OWV * g, q4,
+                                         smem + OFF_DQ + warp_slot + C::STG_DK);
                         bulk_commit();
                     }
                 }
@@ -627,28 +646,37 @@ __global__ void __launch_bounds__(THREADS, 1) bwd_kernel(const __grid_constant__
     }
 }
 
-template <bool F32>
+template <bool F32, int DQK, int DV>
 cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
 {
+    constexpr uint32_t SMEM = BCfg<DQK, DV>::SMEM_BYTES;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(bwd_kernel<F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(bwd_kernel<F32, DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     const int64_t units = static_cast<int64_t>(p.nitems) * p.batch;
     if (units == 0) return cudaSuccess;
     const int64_t cap = sm_count();
-    bwd_kernel<F32><<<static_cast<unsigned>(units < cap ? units : cap), THREADS, SMEM_BYTES, s>>>(p);
+    bwd_kernel<F32, DQK, DV><<<static_cast<unsigned>(units < cap ? units : cap), THREADS, SMEM, s>>>(p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s)
+bool bwd_widths_supported(int dqk, int dv)
 {
-    return f32 ? launch_bwd_t<true>(p, s) : launch_bwd_t<false>(p, s);
+    return (dqk == 64 && dv == 64) || (dqk == 32 && dv == 32) || (dqk == 64 && dv == 128);
+}
+
+cudaError_t launch_bwd(const BwdParams &p, bool f32, int dqk, int dv, cudaStream_t s)
+{
+    if (f32) return dqk == 64 && dv == 64 ? launch_bwd_t<true, 64, 64>(p, s) : cudaErrorInvalidValue;
+    if (dqk == 64 && dv == 64) return launch_bwd_t<false, 64, 64>(p, s);
+    if (dqk == 32 && dv == 32) return launch_bwd_t<false, 32, 32>(p, s);
+    if (dqk == 64 && dv == 128) return launch_bwd_t<false, 64, 128>(p, s);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace st

@@ -108,10 +108,12 @@ int sm_count();
 cudaError_t launch_fwd(const FwdParams &p, bool split, int dqk, int dv, cudaStream_t s);
 cudaError_t launch_fwd_bf16(const FwdParams &p, int dqk, int dv, cudaStream_t s);
 bool fwd_bf16_widths_supported(int dqk, int dv);
-cudaError_t launch_bwd(const BwdParams &p, bool f32, cudaStream_t s);
-cudaError_t launch_bwd_pre(const PreParams &p, bool f32, cudaStream_t s);
-cudaError_t launch_dq_convert(const ConvParams &p, bool f32, cudaStream_t s);
+// Backward row widths (query-key dqk, value dv): bf16 (64, 64), (32, 32), (64, 128); fp32 I/O (64, 64).
+bool bwd_widths_supported(int dqk, int dv);
+cudaError_t launch_bwd(const BwdParams &p, bool f32, int dqk, int dv, cudaStream_t s);
+cudaError_t launch_bwd_pre(const PreParams &p, bool f32, int dqk, int dv, cudaStream_t s);
+cudaError_t launch_dq_convert(const ConvParams &p, bool f32, int dqk, cudaStream_t s);
 cudaError_t launch_split(const SplitParams &p, cudaStream_t s);
-cudaError_t launch_split_finish(const SplitFinishParams &p, bool f32, cudaStream_t s);
+cudaError_t launch_split_finish(const SplitFinishParams &p, bool f32, int dqk, int dv, cudaStream_t s);
 
 }  // namespace st

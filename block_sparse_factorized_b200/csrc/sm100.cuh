@@ -267,6 +267,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "r"(taddr));
 }
 
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// 32 lanes x N consecutive 32-bit columns, N = 8, 16 or 32.
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N])
+{
+    static_assert(N == 8 || N == 16 || N == 32, "columns per load");
+    if constexpr (N == 8) tmem_ld8(taddr, r);
+    else if constexpr (N == 16) tmem_ld16(taddr, r);
+    else tmem_ld32(taddr, r);
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
 {
     asm volatile(
@@ -371,6 +390,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr)
+                 : "memory");
+    return r;
+}
+
 // Byte offset of logical 16-byte chunk `ch` (0..1) of row `r` in a 32-byte-swizzled tile
 // (32-byte rows; chunk index XOR bit 2 of the row).
 __device__ __forceinline__ uint32_t sw32_off(uint32_t r, uint32_t ch)
@@ -389,6 +416,18 @@ __device__ __forceinline__ uint32_t sw64_off(uint32_t r, uint32_t ch)
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t ch)
 {
     return r * 128u + ((ch ^ (r & 7u)) << 4);
+}
+
+// Byte offset of 16-byte chunk `ch` of row `r` in a tile of SPAN-byte rows written with the
+// matching TMA swizzle (none for 16-byte rows, else the SPAN-byte swizzle).
+template <int SPAN>
+__device__ __forceinline__ uint32_t swz_off(uint32_t r, uint32_t ch)
+{
+    static_assert(SPAN == 16 || SPAN == 32 || SPAN == 64 || SPAN == 128, "row span");
+    if constexpr (SPAN == 16) return r * 16u;
+    else if constexpr (SPAN == 32) return sw32_off(r, ch);
+    else if constexpr (SPAN == 64) return sw64_off(r, ch);
+    else return sw128_off(r, ch);
 }
 
 }  // namespace st

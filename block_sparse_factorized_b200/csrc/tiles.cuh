@@ -136,6 +136,44 @@ __device__ __forceinline__ void store_warp_slice(const FrameMaps &m, int32_t fr,
     }
 }
 
+// Per-width tile geometry.  A 128-row bf16 tile of W columns is loaded as NBOX TMA boxes of BOX
+// columns, each one swizzle span wide (64-byte swizzle for W = 32, 128-byte otherwise), stored
+// one after another: box b holds columns b*BOX .. b*BOX + BOX - 1 of every row.
+template <int W>
+struct Tile {
+    static_assert(W == 32 || W == 64 || W == 128, "row width");
+    static constexpr int BOX = W < 64 ? W : 64;
+    static constexpr int NBOX = W / BOX;
+    static constexpr uint32_t SPAN = BOX * 2;                // bytes per row of a box (swizzle span)
+    static constexpr uint32_t BOX_BYTES = 128 * SPAN;
+    static constexpr uint32_t BYTES = NBOX * BOX_BYTES;
+    static constexpr uint32_t LAYOUT = W < 64 ? UMMA_SW64 : UMMA_SW128;
+    // K-major operand (rows = M or N, K = the W columns): the K16 step k starts 32 bytes further
+    // in the same box, or in the next box once a box's columns are used up; 8-row groups are
+    // 8 * SPAN bytes apart.
+    __device__ static uint64_t kmajor(uint32_t base, int k)
+    {
+        const int col = 16 * k;
+        return desc_swz(base + (col / BOX) * BOX_BYTES + (col % BOX) * 2, 16, 8 * SPAN, LAYOUT);
+    }
+    // MN-major operand (K = the 128 rows, N = the W columns): the K16 step k starts 16 rows
+    // further; 8-row groups are 8 * SPAN bytes apart (SBO) and the N atoms are the boxes (LBO).
+    __device__ static uint64_t mnmajor(uint32_t base, int k)
+    {
+        return desc_swz(base + 16 * k * SPAN, BOX_BYTES, 8 * SPAN, LAYOUT);
+    }
+};
+
+// TMA load of tile t of frame fr of batch-head bh into dst: NBOX boxes, one transaction count.
+template <int W>
+__device__ __forceinline__ void load_tile_w(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o, int32_t t,
+                                            int32_t bh, uint8_t *dst, uint64_t *bar)
+{
+#pragma unroll
+    for (int b = 0; b < Tile<W>::NBOX; ++b)
+        load_tile_x(m, fr, g, o, t, bh, b * Tile<W>::BOX, dst + b * Tile<W>::BOX_BYTES, bar);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 

@@ -77,10 +77,10 @@ def test_argument_errors():
     d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
     assert lib.st_attn_fwd(fake, fake, fake, lay.handle, fake, fake, None, 0, ctypes.byref(d), None) == 4
     # row widths (query-key d, value dv; dv = 0 means d): the bf16 forward takes (32, 32),
-    # (64, 64), (128, 128) and (64, 128) -- those pass the width check and meet NOT_UPLOADED --
-    # the backward and fp32 I/O only (64, 64); other widths are valid but unsupported, a negative
-    # value width is invalid
-    for dqk, dv, dt, fwd_want, bwd_want in ((32, 0, 1, 4, 2), (128, 0, 1, 4, 2), (64, 128, 1, 4, 2),
+    # (64, 64), (128, 128) and (64, 128), the bf16 backward (32, 32), (64, 64) and (64, 128) --
+    # those pass the width check and meet NOT_UPLOADED -- fp32 I/O only (64, 64); other widths
+    # are valid but unsupported, a negative value width is invalid
+    for dqk, dv, dt, fwd_want, bwd_want in ((32, 0, 1, 4, 4), (128, 0, 1, 4, 2), (64, 128, 1, 4, 4),
                                             (64, 64, 1, 4, 4), (64, 0, 2, 4, 4), (32, 0, 2, 2, 2),
                                             (48, 0, 1, 2, 2), (64, 32, 1, 2, 2), (256, 0, 1, 2, 2),
                                             (64, -1, 1, 1, 1)):

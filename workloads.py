@@ -65,6 +65,9 @@ WORKLOADS = {
                                            128, 0, 2, 16),
     "strided_n65536_l256": Workload("strided_n65536_l256", STRIDED, ALTERNATING, 65536, 256, 0,
                                     1, 8),
+    # the 64x64x3 raster at the image model's own head width: 16 heads of 512 / 16 = 32
+    "strided_n12288_l128_d32": Workload("strided_n12288_l128_d32", STRIDED, ALTERNATING, 12288, 128, 0,
+                                        2, 16, d=32),
     # the text model's own setting: fixed pattern with merged heads (each head reads its block and
     # every earlier block's summary run), n = 12288, l = 128, c = 32, 8 heads
     "fixed_merged_n12288_l128_c32": Workload("fixed_merged_n12288_l128_c32", FIXED, MERGED, 12288,
