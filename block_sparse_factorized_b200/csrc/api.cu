@@ -511,7 +511,9 @@ size_t st_attn_decode_workspace_bytes(const st_desc_t *desc, const st_layout_t *
     if (!desc || !layout || !sizes_valid(desc)) return 0;
     const size_t nsplit = static_cast<size_t>((desc->n + st::DEC_CHUNK - 1) / st::DEC_CHUNK);
     const size_t part = static_cast<size_t>(value_width(desc)) + 4;  // dec_part(dv) floats per chunk
-    return round256(static_cast<size_t>(desc->batch) * desc->heads * nsplit * part * sizeof(float));
+    const size_t bh = static_cast<size_t>(desc->batch) * desc->heads;
+    // the per-(batch, head) chunk counters, then the chunk results
+    return round256(bh * sizeof(int32_t)) + round256(bh * nsplit * part * sizeof(float));
 }
 
 st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cache, const st_layout_t *layout,
@@ -538,7 +540,9 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     p.v = v_cache;
     p.o = o;
     p.lse = lse;
-    p.part = static_cast<float *>(workspace);
+    const size_t bh = static_cast<size_t>(desc->batch) * desc->heads;
+    p.cnt = static_cast<int32_t *>(workspace);
+    p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) + round256(bh * sizeof(int32_t)));
     int64_t most = 1;
     for (int32_t h = 0; h < desc->heads; ++h) {
         p.kind[h] = L.head_kind[h];
@@ -555,6 +559,7 @@ st_status_t st_attn_decode(const void *q, const void *k_cache, const void *v_cac
     p.scale_log2 = LOG2E / sqrtf(static_cast<float>(desc->d));  // log2(e) / sqrt(d)
     const int64_t nsplit = (most + st::DEC_CHUNK - 1) / st::DEC_CHUNK;
     if (nsplit > 65535) return ST_ERR_UNSUPPORTED;  // grid dimension y: a row with over 4 M allowed keys
+    if (cudaMemsetAsync(p.cnt, 0, bh * sizeof(int32_t), stream) != cudaSuccess) return ST_ERR_CUDA;
     return st::launch_decode(p, static_cast<int32_t>(nsplit), desc->dtype == ST_FP32, static_cast<int>(desc->d),
                              static_cast<int>(dv), stream) == cudaSuccess
                ? ST_OK

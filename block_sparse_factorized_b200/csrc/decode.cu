@@ -14,8 +14,9 @@
 // threads works as 16 groups of 8 lanes, a group taking 4 keys with each lane holding an eighth of
 // the query-key row (d / 8 components) and of the value row (dv / 8).  All K and V loads of a chunk
 // are issued before any is used (the work is one round trip to memory, not a chain of them); then
-// scores, their maximum and 2^(s - M) v.  Each CTA leaves (M, L, O) of its chunk in the workspace; a
-// second kernel combines the chunks of a (batch, head) by log-sum-exp weights.
+// scores, their maximum and 2^(s - M) v.  Each CTA leaves (M, L, O) of its chunk in the workspace and
+// counts itself in the (batch, head)'s counter; the CTA that completes the count combines the
+// chunks by log-sum-exp weights -- one launch per step, the counters zeroed before it.
 #include "decode.h"
 #include "tiles.cuh"
 
@@ -123,41 +124,75 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_kernel(const DecodeParams 
     for (int t = 0; t < NV; ++t) red[grp][NV * l8 + t] = acc[t];
     if (l8 == 0) red[grp][DV] = lsum;
     __syncthreads();
-    float *part = p.part + (static_cast<size_t>(bh) * gridDim.y + blockIdx.y) * PART;
+    const int32_t nsplit = static_cast<int32_t>(gridDim.y);
+    float *parts = p.part + static_cast<size_t>(bh) * nsplit * PART;
+    float *part = parts + static_cast<size_t>(blockIdx.y) * PART;
     for (int c = threadIdx.x; c < DV + 1; c += DEC_THREADS) {
         float sum = 0.f;
         for (int g = 0; g < DEC_GROUPS; ++g) sum += red[g][c];  // fixed order
-        part[2 + c] = sum;  // O (DV columns) then L
+        part[c < DV ? 4 + c : 1] = sum;  // O (DV columns, 16-byte aligned at 4) and L at 1
     }
     if (threadIdx.x == 0) part[0] = M;  // -inf for a chunk without keys
-}
-
-// One (batch, head) per CTA, one output column per thread: O = sum_c 2^(M_c - M) O_c / L,
-// L = sum_c 2^(M_c - M) L_c, lse = (M + log2 L) ln 2; a row without keys gets O = 0, lse = -inf.
-template <bool F32, int DV>
-__global__ void __launch_bounds__(DV) decode_combine_kernel(const DecodeParams p, int32_t nsplit)
-{
-    constexpr int PART = dec_part(DV);
-    const int32_t bh = blockIdx.x, t = threadIdx.x;
-    const float *part = p.part + static_cast<size_t>(bh) * nsplit * PART;
-    float M = -INFINITY;
-    for (int c = 0; c < nsplit; ++c) M = fmaxf(M, part[c * PART]);
-    float L = 0.f, o = 0.f;
-    if (M != -INFINITY)
-        for (int c = 0; c < nsplit; ++c) {
-            const float mc = part[c * PART];
-            const float w = mc == -INFINITY ? 0.f : ex2(mc - M);
-            L = fmaf(w, part[c * PART + 2 + DV], L);
-            o = fmaf(w, part[c * PART + 2 + t], o);
+    // count this chunk; the CTA that brings the count to nsplit combines (the fences order every
+    // CTA's part before its count, and the counts before the combining CTA's reads)
+    __shared__ int32_t is_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&p.cnt[bh], 1) == nsplit - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // O = sum_c 2^(M_c - M) O_c / L, L = sum_c 2^(M_c - M) L_c, lse = (M + log2 L) ln 2; a row
+    // without keys gets O = 0, lse = -inf.  The parts are read through L2 (ld.global.cg: other CTAs
+    // wrote them), spread over all threads so that each makes few independent loads: thread
+    // (group g, quad q) adds, for the chunks c = g, g + G, ..., their weighted columns 4qd .. 4qd + 3
+    // (and, for qd = 0, their L); the G group sums are then added in group order (deterministic).
+    constexpr int NQD = DV / 4;                 // 16-byte quads of a value row
+    constexpr int G = DEC_THREADS / NQD;        // chunk groups
+    __shared__ float osum[G][DV + 1];
+    float mloc = -INFINITY;
+    for (int c = threadIdx.x; c < nsplit; c += DEC_THREADS) mloc = fmaxf(mloc, __ldcg(parts + c * PART));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mloc;
+    __syncthreads();
+    const float Mall = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    const int g = threadIdx.x / NQD, qd = threadIdx.x % NQD;
+    float4 oq = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lacc = 0.f;
+    if (Mall != -INFINITY)
+        for (int c = g; c < nsplit; c += G) {
+            const float *pc = parts + static_cast<size_t>(c) * PART;
+            const float mc = __ldcg(pc);
+            const float4 x = __ldcg(reinterpret_cast<const float4 *>(pc + 4) + qd);
+            const float w = mc == -INFINITY ? 0.f : ex2(mc - Mall);
+            oq.x = fmaf(w, x.x, oq.x);
+            oq.y = fmaf(w, x.y, oq.y);
+            oq.z = fmaf(w, x.z, oq.z);
+            oq.w = fmaf(w, x.w, oq.w);
+            if (qd == 0) lacc = fmaf(w, __ldcg(pc + 1), lacc);
         }
-    const bool has = L > 0.f;
-    o = has ? o / L : 0.f;
-    if (F32)
-        static_cast<float *>(p.o)[static_cast<size_t>(bh) * DV + t] = o;
-    else
-        static_cast<uint16_t *>(p.o)[static_cast<size_t>(bh) * DV + t] =
-            static_cast<uint16_t>(pack_bf16(o, 0.f) & 0xFFFFu);
-    if (t == 0) p.lse[bh] = has ? (M + lg2(L)) * LN2 : -INFINITY;
+    osum[g][4 * qd] = oq.x;
+    osum[g][4 * qd + 1] = oq.y;
+    osum[g][4 * qd + 2] = oq.z;
+    osum[g][4 * qd + 3] = oq.w;
+    if (qd == 0) osum[g][DV] = lacc;
+    __syncthreads();
+    for (int t = threadIdx.x; t < DV; t += DEC_THREADS) {
+        float L = 0.f, o = 0.f;
+        for (int gg = 0; gg < G; ++gg) {  // fixed order
+            L += osum[gg][DV];
+            o += osum[gg][t];
+        }
+        const bool has = L > 0.f;
+        o = has ? o / L : 0.f;
+        if (F32)
+            static_cast<float *>(p.o)[static_cast<size_t>(bh) * DV + t] = o;
+        else
+            static_cast<uint16_t *>(p.o)[static_cast<size_t>(bh) * DV + t] =
+                static_cast<uint16_t>(pack_bf16(o, 0.f) & 0xFFFFu);
+        if (t == 0) p.lse[bh] = has ? (Mall + lg2(L)) * LN2 : -INFINITY;
+    }
 }
 
 template <bool F32, int D, int DV>
@@ -165,7 +200,6 @@ cudaError_t launch_w(const DecodeParams &p, int32_t nsplit, cudaStream_t s)
 {
     const dim3 grid(static_cast<unsigned>(p.bh), static_cast<unsigned>(nsplit));
     decode_kernel<F32, D, DV><<<grid, DEC_THREADS, 0, s>>>(p);
-    decode_combine_kernel<F32, DV><<<static_cast<unsigned>(p.bh), DV, 0, s>>>(p, nsplit);
     return cudaGetLastError();
 }
 

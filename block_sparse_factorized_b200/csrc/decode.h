@@ -8,7 +8,7 @@
 namespace st {
 
 constexpr int DEC_CHUNK = 64;   // keys per CTA (16 groups x 4 keys)
-// floats per chunk result for value rows of width dv: M, (unused), O[dv], L, (pad)
+// floats per chunk result for value rows of width dv: M, L, (pad, pad), O[dv] -- O 16-byte aligned
 __host__ __device__ constexpr int dec_part(int dv) { return dv + 4; }
 
 // Allowed keys of one row: nu runs, run u covering g0 + u * gs .. + glen - 1 (the last run cut to
@@ -91,6 +91,7 @@ struct DecodeParams {
     void *o;            // [B*H, dv]
     float *lse;         // [B*H], natural log
     float *part;        // [B*H, nsplit, dec_part(dv)] chunk results (workspace)
+    int32_t *cnt;       // [B*H] chunks finished (workspace, zero before the launch)
     int32_t kind[64], off[64];
     int64_t pos, n, l, c;
     int32_t bh, heads;

@@ -277,7 +277,10 @@ ST_API st_status_t st_attn_bwd_noalloc(const void *q, const void *k, const void 
  *             not read
  *   o:        [batch, heads, 64] output (desc->dtype);  lse: [batch, heads] fp32 output (natural
  *             log; -inf for a row with no allowed key, whose o is 0)
- *   workspace: st_attn_decode_workspace_bytes (per-chunk partial results), 256-byte aligned
+ *   workspace: st_attn_decode_workspace_bytes (a chunk counter per (batch, head), then the per-chunk
+ *             partial results), 256-byte aligned; the call zeroes the counters (one memset on
+ *             `stream`) and launches one kernel, whose last chunk of each row combines the row's
+ *             chunks, so calls that share a workspace must not overlap on the GPU
  * desc is the full-sequence descriptor (its n is the cache capacity).  The layout need not be
  * uploaded: the kernels read only the per-head set kinds, passed by value.  Errors:
  * ST_ERR_INVALID_ARG (NULL pointers, pos outside [0, n), heads or n not the layout's),

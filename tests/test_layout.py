@@ -126,9 +126,10 @@ def test_decode_argument_errors():
     lay = bsf.Layout(S, A, 2, 256, 16)
     fake, odd = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
     d = _abi.st_desc_t(1, 2, 256, 64, 1, 0)
-    # 256 rows of cache -> 4 chunks of 64 keys, 68 floats each, per (batch, head), rounded to 256 B
+    # a chunk counter per (batch, head) (256 B after rounding), then 256 rows of cache -> 4 chunks of
+    # 64 keys, 68 floats each, per (batch, head), rounded to 256 B
     need = lib.st_attn_decode_workspace_bytes(ctypes.byref(d), lay.handle)
-    assert need == 2304
+    assert need == 256 + 2304
     ws = ctypes.c_void_p(1 << 24)
 
     def call(q=fake, pos=100, desc=d, w=ws, wb=need):
@@ -143,7 +144,7 @@ def test_decode_argument_errors():
     assert call(desc=_abi.st_desc_t(1, 2, 256, 64, 1, -1)) == 1   # negative value width
     # the chunk record is dv + 4 floats: 2 x 4 x 132 x 4 bytes at dv = 128
     wide = _abi.st_desc_t(1, 2, 256, 64, 1, 128)
-    assert lib.st_attn_decode_workspace_bytes(ctypes.byref(wide), lay.handle) == 4352
+    assert lib.st_attn_decode_workspace_bytes(ctypes.byref(wide), lay.handle) == 256 + 4352
     assert call(desc=wide) == 8                                  # the 64-wide workspace is too small
     assert call(q=odd) == 3                       # misaligned
     assert call(w=None) == 8 and call(wb=need - 1) == 8          # workspace missing / too small
