@@ -27,44 +27,6 @@
 namespace st {
 namespace {
 
-// Per-width tile geometry.  A 128-row bf16 tile of W columns is loaded as NBOX TMA boxes of BOX
-// columns, each one swizzle span wide (64-byte swizzle for W = 32, 128-byte otherwise), stored
-// one after another: box b holds columns b*BOX .. b*BOX + BOX - 1 of every row.
-template <int W>
-struct Tile {
-    static_assert(W == 32 || W == 64 || W == 128, "row width");
-    static constexpr int BOX = W < 64 ? W : 64;
-    static constexpr int NBOX = W / BOX;
-    static constexpr uint32_t SPAN = BOX * 2;                // bytes per row of a box (swizzle span)
-    static constexpr uint32_t BOX_BYTES = 128 * SPAN;
-    static constexpr uint32_t BYTES = NBOX * BOX_BYTES;
-    static constexpr uint32_t LAYOUT = W < 64 ? UMMA_SW64 : UMMA_SW128;
-    // K-major operand (rows = M or N, K = the W columns): the K16 step k starts 32 bytes further
-    // in the same box, or in the next box once a box's columns are used up; 8-row groups are
-    // 8 * SPAN bytes apart.
-    __device__ static uint64_t kmajor(uint32_t base, int k)
-    {
-        const int col = 16 * k;
-        return desc_swz(base + (col / BOX) * BOX_BYTES + (col % BOX) * 2, 16, 8 * SPAN, LAYOUT);
-    }
-    // MN-major operand (K = the 128 rows, N = the W columns): the K16 step k starts 16 rows
-    // further; 8-row groups are 8 * SPAN bytes apart (SBO) and the N atoms are the boxes (LBO).
-    __device__ static uint64_t mnmajor(uint32_t base, int k)
-    {
-        return desc_swz(base + 16 * k * SPAN, BOX_BYTES, 8 * SPAN, LAYOUT);
-    }
-};
-
-// TMA load of tile t of frame fr of batch-head bh into dst: NBOX boxes, one transaction count.
-template <int W>
-__device__ __forceinline__ void load_tile_w(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o, int32_t t,
-                                            int32_t bh, uint8_t *dst, uint64_t *bar)
-{
-#pragma unroll
-    for (int b = 0; b < Tile<W>::NBOX; ++b)
-        load_tile_x(m, fr, g, o, t, bh, b * Tile<W>::BOX, dst + b * Tile<W>::BOX_BYTES, bar);
-}
-
 constexpr int NST = 2;                         // K/V ring depth
 constexpr int NQB = 2;                         // Q buffers
 constexpr int NSCHED = 4;                      // claimed-unit ring depth
@@ -84,7 +46,10 @@ struct Cfg {
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + NQB * QB;
     static constexpr uint32_t OFF_V = OFF_K + NST * QB;
-    static constexpr uint32_t OFF_BAR = OFF_V + NST * VB;
+    // a merge epilogue's per-warp staging of its 32 output rows (DV * 2 bytes each)
+    static constexpr uint32_t OFF_STG = OFF_V + NST * VB;
+    static constexpr uint32_t STG_ROW = DV * 2;
+    static constexpr uint32_t OFF_BAR = OFF_STG + 4 * 32 * STG_ROW;
     static constexpr uint32_t OFF_UNITS = OFF_BAR + 256;
     static constexpr uint32_t SMEM_BYTES = OFF_UNITS + 4 * 96;
     static_assert(SMEM_BYTES * CTAS_PER_SM <= 228 * 1024 - CTAS_PER_SM * 1024, "shared memory per SM");
@@ -398,29 +363,73 @@ __global__ void __launch_bounds__(THREADS, (Cfg<DQK, DV>::CTAS_PER_SM)) fwd_bf16
                     lse2 = Lm + lg2(tot);
                 }
             }
-            if (e.i < 0 || *abort != 0) return;  // grid-frame padding row
-            // 8 columns (16 bytes) at a time; a merge reads each 16 bytes of the first pass's row
-            // before it overwrites them
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.o_prev + rowoff * DV);
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + rowoff * DV);
+            const bool live = e.i >= 0 && *abort == 0;  // not a grid-frame padding row
+            if (!__any_sync(0xffffffffu, cprev != 0.f)) {
+                // no first-pass output to fold in: 8 columns (16 bytes) at a time, row by row
+                if (live) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.o + rowoff * DV);
+#pragma unroll
+                    for (int q = 0; q < DV / 8; ++q) {
+                        float a[8];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) a[c] = has_o ? cnew * __uint_as_float(v[8 * q + c]) : 0.f;
+                        dst[q] = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                                            pack_bf16(a[6], a[7]));
+                    }
+                    p.lse[rowoff] = lse2 * LN2;
+                }
+                return;
+            }
+            // A merge: the warp's 32 rows go through its shared staging, so that the first pass's
+            // rows are read whole (a warp instruction reads RPI complete rows of DV * 2 bytes, not
+            // 16 bytes of each of 32 rows scattered over the grid frame) and written back whole.
+            // Chunk c (16 bytes) of staged row r sits at stg_off(r, c), swizzled so that both
+            // access patterns are free of bank conflicts.
+            constexpr int CPR = DV / 8;                 // 16-byte chunks per row
+            constexpr int RPI = 32 / CPR;               // rows per warp instruction
+            const uint32_t stg = smem_u32(smem + C::OFF_STG) + q4 * 32 * C::STG_ROW;
+            auto stg_off = [&](uint32_t r, uint32_t c) {
+                return CPR >= 8 ? r * C::STG_ROW + ((c ^ (r & 7u)) << 4) : sw64_off(r, c);
+            };
+            const int32_t sub_row = lane / CPR, sub_c = lane % CPR;
+#pragma unroll
+            for (int r0 = 0; r0 < 32; r0 += RPI) {
+                const int32_t r = r0 + sub_row;
+                const int32_t ir = __shfl_sync(0xffffffffu, live ? e.i : -1, r);
+                uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                if (ir >= 0)
+                    x = reinterpret_cast<const uint4 *>(p.o_prev + (static_cast<size_t>(e.bh) * p.g.n + ir) * DV)[sub_c];
+                st_shared_v4(stg + stg_off(r, sub_c), x.x, x.y, x.z, x.w);
+            }
+            __syncwarp();
+            // this thread's row: O / l plus the first pass's share, as bf16, into the staging
 #pragma unroll
             for (int q = 0; q < DV / 8; ++q) {
                 float a[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) a[c] = has_o ? cnew * __uint_as_float(v[8 * q + c]) : 0.f;
-                if (cprev != 0.f) {
-                    const uint4 x = src[q];
-                    const uint32_t pw[4] = {x.x, x.y, x.z, x.w};
+                const uint4 x = ld_shared_v4(stg + stg_off(lane, q));
+                const uint32_t pw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        a[2 * c] = fmaf(cprev, bf16_lo(pw[c]), a[2 * c]);
-                        a[2 * c + 1] = fmaf(cprev, bf16_hi(pw[c]), a[2 * c + 1]);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    a[2 * c] = fmaf(cprev, bf16_lo(pw[c]), a[2 * c]);
+                    a[2 * c + 1] = fmaf(cprev, bf16_hi(pw[c]), a[2 * c + 1]);
                 }
-                dst[q] = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
-                                    pack_bf16(a[6], a[7]));
+                st_shared_v4(stg + stg_off(lane, q), pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                             pack_bf16(a[6], a[7]));
             }
-            p.lse[rowoff] = lse2 * LN2;
+            __syncwarp();
+            // whole rows to global memory (rows of the grid frame's padding are skipped)
+#pragma unroll
+            for (int r0 = 0; r0 < 32; r0 += RPI) {
+                const int32_t r = r0 + sub_row;
+                const int32_t ir = __shfl_sync(0xffffffffu, live ? e.i : -1, r);
+                const uint4 x = ld_shared_v4(stg + stg_off(r, sub_c));
+                if (ir >= 0)
+                    reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(e.bh) * p.g.n + ir) * DV)[sub_c] = x;
+            }
+            __syncwarp();  // the staging is reused by this warp's next epilogue
+            if (live) p.lse[rowoff] = lse2 * LN2;
         };
         for (int32_t j = 0; ok; ++j) {
             Unit U;

@@ -71,20 +71,6 @@ __device__ __forceinline__ void load_tile(const FrameMaps &m, int32_t fr, const 
     load_tile_x(m, fr, g, o, t, bh, 0, dst, bar);
 }
 
-// L2 prefetch of tile t of frame fr (same coordinates as load_tile).
-__device__ __forceinline__ void prefetch_tile(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
-                                              int32_t t, int32_t bh)
-{
-    if (fr == FR_NAT) {
-        tma_prefetch_l2_3d(&m.nat, 0, t * TILE, bh);
-    } else if (fr == FR_COL) {
-        const int32_t grp = fdiv(t, g.div_tpc), rt = t - grp * g.tpc;
-        tma_prefetch_l2_4d(&m.col, 0, rt * TILE, grp * g.cpt, bh);
-    } else {
-        tma_prefetch_l2_4d(&m.sum, 0, g.l - g.c - o, t * g.upt, bh);
-    }
-}
-
 // TMA store of a 16 KB tile; rows outside the tensor (padding of the grid and summary frames)
 // are clipped by the copy engine.
 __device__ __forceinline__ void store_tile(const FrameMaps &m, int32_t fr, const Geom &g, int32_t o,
