@@ -94,3 +94,9 @@ def test_decode_widths(w, d, dv):
 def test_decode_widths_fp32(d, dv):
     """fp32 I/O at the other widths (the forward has no fp32 kernel there: oracle only)."""
     run_case(FP32[0].with_(d=d, dv=dv), with_fwd=False)
+
+
+def test_decode_long_rows():
+    """Long rows: a fixed summary head at n = 2^18 has up to 65,664 allowed keys, over a thousand
+    64-key chunks of one row, combined through the workspace by the row's last chunk."""
+    run_case(Workload("f_alt_n262144_l128_c32", FIXED, ALTERNATING, 1 << 18, 128, 32, 1, 2))
